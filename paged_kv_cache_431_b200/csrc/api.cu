@@ -1,0 +1,367 @@
+// api.cu -- the C-ABI of libpkv: argument validation, pool handles, tensor maps,
+// workspace layout and kernel launches.  Every entry point validates on the host
+// before launching and returns a PKV_* status; nothing here synchronizes except
+// pkv_read_device_status.
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+namespace pkv {
+
+int row_bytes_of(int dtype, int head_dim)
+{
+    switch (dtype) {
+    case PKV_F16:
+    case PKV_BF16: return 2 * head_dim;
+    case PKV_INT8:
+    case PKV_FP8E4M3: return head_dim;
+    case PKV_INT4: return head_dim / 2;
+    default: return -1;
+    }
+}
+
+bool is_quantized(int dtype) { return dtype == PKV_INT8 || dtype == PKV_INT4 || dtype == PKV_FP8E4M3; }
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// One layer's K or V pool as a 2-D tensor [N * H_kv * 16 rows][row elements], loaded in
+// boxes of 16 rows x (at most) 128 bytes with the matching shared-memory swizzle.
+static bool make_map(CUtensorMap* map, void* base, const pkv_pool_desc& d, int row_bytes)
+{
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const bool b16 = d.kv_dtype == PKV_F16 || d.kv_dtype == PKV_BF16;
+    const int esize = b16 ? 2 : 1;
+    const cuuint64_t dims[2] = {(cuuint64_t)(row_bytes / esize), (cuuint64_t)d.num_blocks * d.num_kv_heads * PKV_BLOCK_SIZE};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    const int box_bytes = row_bytes < 128 ? row_bytes : 128;
+    const cuuint32_t box[2] = {(cuuint32_t)(box_bytes / esize), (cuuint32_t)PKV_BLOCK_SIZE};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle swz = box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : box_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = enc(map, b16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtensorMap** tmv)
+{
+    std::lock_guard<std::mutex> lock(pool->mu);
+    if (!pool->maps_ready) {
+        const int L = pool->d.num_layers;
+        pool->tmk.resize(L);
+        pool->tmv.resize(L);
+        for (int l = 0; l < L; ++l) {
+            uint8_t* kb = static_cast<uint8_t*>(pool->d.k_data) + (size_t)l * pool->layer_bytes;
+            uint8_t* vb = static_cast<uint8_t*>(pool->d.v_data) + (size_t)l * pool->layer_bytes;
+            if (!make_map(&pool->tmk[l], kb, pool->d, pool->row_bytes) ||
+                !make_map(&pool->tmv[l], vb, pool->d, pool->row_bytes))
+                return PKV_ERR_CUDA;
+        }
+        pool->maps_ready = true;
+    }
+    *tmk = &pool->tmk[layer];
+    *tmv = &pool->tmv[layer];
+    return PKV_OK;
+}
+
+// Split-K partition size: 512 tokens unless the batch is too small to fill the GPU
+// with one-warp CTAs, then down to 128.
+static int choose_partition(int B, int H_kv, int max_ctx, const pkv_decode_opts* o)
+{
+    if (o && o->partition_tokens > 0) return o->partition_tokens;
+    const long target = 4L * num_sms() * 8;
+    int P = 512;
+    while (P > 128) {
+        const long parts = (max_ctx + P - 1) / P;
+        if ((long)B * H_kv * (parts > 0 ? parts : 1) >= target) break;
+        P /= 2;
+    }
+    return P;
+}
+
+static bool valid_partition(int P) { return P >= 64 && P <= 4096 && P % PKV_BLOCK_SIZE == 0; }
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+int pkv_version(void) { return 100; }
+
+const char* pkv_strerror(int status)
+{
+    switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_NULL: return "a required pointer is NULL";
+    case PKV_ERR_ARG: return "an argument is out of range";
+    case PKV_ERR_DTYPE: return "unsupported dtype or dtype combination";
+    case PKV_ERR_SHAPE: return "inconsistent sizes";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_CUDA: return "a CUDA call failed";
+    case PKV_ERR_TIMEOUT: return "a kernel gave up waiting on a bulk copy";
+    case PKV_ERR_INDEX: return "the device saw a block id, slot or context length out of range";
+    case PKV_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    default: return "unknown status";
+    }
+}
+
+static int validate_desc(const pkv_pool_desc* d)
+{
+    if (!d) return PKV_ERR_NULL;
+    if (d->num_layers <= 0 || d->num_blocks <= 0 || d->num_kv_heads <= 0) return PKV_ERR_ARG;
+    if (d->block_size != PKV_BLOCK_SIZE) return PKV_ERR_ARG;
+    if (d->head_dim != 64 && d->head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (row_bytes_of(d->kv_dtype, d->head_dim) <= 0) return PKV_ERR_DTYPE;
+    if ((long long)d->num_blocks * d->num_kv_heads * PKV_BLOCK_SIZE > 0x7fffffffLL) return PKV_ERR_ARG;
+    return PKV_OK;
+}
+
+size_t pkv_pool_bytes(const pkv_pool_desc* d, size_t* scale_bytes)
+{
+    if (scale_bytes) *scale_bytes = 0;
+    if (validate_desc(d) != PKV_OK) return 0;
+    const size_t per_layer = (size_t)d->num_blocks * d->num_kv_heads * PKV_BLOCK_SIZE * row_bytes_of(d->kv_dtype, d->head_dim);
+    if (scale_bytes && is_quantized(d->kv_dtype))
+        *scale_bytes = (size_t)d->num_layers * d->num_blocks * d->num_kv_heads * sizeof(float);
+    return per_layer * d->num_layers;
+}
+
+int kv_pool_create(const pkv_pool_desc* d, pkv_pool_t* out)
+{
+    if (!out) return PKV_ERR_NULL;
+    *out = nullptr;
+    int rc = validate_desc(d);
+    if (rc != PKV_OK) return rc;
+    if (!d->k_data || !d->v_data) return PKV_ERR_NULL;
+    if (is_quantized(d->kv_dtype) && (!d->k_scale || !d->v_scale)) return PKV_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(d->k_data) | reinterpret_cast<uintptr_t>(d->v_data)) & 15) return PKV_ERR_ARG;
+    pkv_pool* p = new (std::nothrow) pkv_pool();
+    if (!p) return PKV_ERR_ARG;
+    p->d = *d;
+    p->row_bytes = row_bytes_of(d->kv_dtype, d->head_dim);
+    p->tile_bytes = (size_t)PKV_BLOCK_SIZE * p->row_bytes;
+    p->layer_bytes = (size_t)d->num_blocks * d->num_kv_heads * p->tile_bytes;
+    p->layer_scales = is_quantized(d->kv_dtype) ? (size_t)d->num_blocks * d->num_kv_heads : 0;
+    *out = p;
+    return PKV_OK;
+}
+
+int kv_pool_destroy(pkv_pool_t pool)
+{
+    delete pool;
+    return PKV_OK;
+}
+
+size_t kv_append_workspace_bytes(pkv_pool_t pool, int num_tokens)
+{
+    if (!pool || num_tokens < 0) return 0;
+    return append_workspace_bytes(pool->d.num_blocks, pool->d.num_kv_heads, pool->d.kv_dtype);
+}
+
+int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, int src_dtype, const int32_t* slot_mapping,
+              int num_tokens, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!pool) return PKV_ERR_NULL;
+    const pkv_pool_desc& d = pool->d;
+    if (layer < 0 || layer >= d.num_layers || num_tokens < 0) return PKV_ERR_ARG;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping) return PKV_ERR_NULL;
+    if (is_quantized(d.kv_dtype)) {
+        if (src_dtype != PKV_BF16) return PKV_ERR_DTYPE;
+        const size_t need = append_workspace_bytes(d.num_blocks, d.num_kv_heads, d.kv_dtype);
+        if (!workspace || workspace_bytes < need) return PKV_ERR_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(workspace) & 3) return PKV_ERR_ARG;
+    } else if (src_dtype != d.kv_dtype) {
+        return PKV_ERR_DTYPE;
+    }
+    const uintptr_t align = is_quantized(d.kv_dtype) ? 8 : 16;
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & (align - 1)) return PKV_ERR_ARG;
+    if ((long long)num_tokens * d.num_kv_heads > 0x7fffffffLL / 32) return PKV_ERR_ARG;
+    AppendArgs a;
+    a.k = k;
+    a.v = v;
+    a.slots = slot_mapping;
+    a.T = num_tokens;
+    a.N = d.num_blocks;
+    a.H_kv = d.num_kv_heads;
+    a.d = d.head_dim;
+    a.kv_dtype = d.kv_dtype;
+    a.k_pool = static_cast<uint8_t*>(d.k_data) + (size_t)layer * pool->layer_bytes;
+    a.v_pool = static_cast<uint8_t*>(d.v_data) + (size_t)layer * pool->layer_bytes;
+    a.k_scale = d.k_scale ? d.k_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.v_scale = d.v_scale ? d.v_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.workspace = workspace;
+    a.status = d.device_status;
+    return launch_append(a, static_cast<cudaStream_t>(stream));
+}
+
+static int decode_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, const pkv_decode_opts* opts, int* P,
+                               int* max_parts)
+{
+    *P = choose_partition(num_seqs, pool->d.num_kv_heads, max_ctx, opts);
+    if (!valid_partition(*P)) return PKV_ERR_ARG;
+    *max_parts = max_ctx > 0 ? (max_ctx + *P - 1) / *P : 1;
+    return PKV_OK;
+}
+
+size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_context_len,
+                                    const pkv_decode_opts* opts)
+{
+    if (!pool || num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return 0;
+    int P, parts;
+    if (decode_partitioning(pool, num_seqs, max_context_len, opts, &P, &parts) != PKV_OK) return 0;
+    if (parts <= 1) return 0;
+    return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float);
+}
+
+int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, const int32_t* block_tables,
+                      int block_table_width, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                      int max_context_len, float scale, float* out, void* workspace, size_t workspace_bytes,
+                      const pkv_decode_opts* opts, void* stream)
+{
+    if (!pool) return PKV_ERR_NULL;
+    const pkv_pool_desc& d = pool->d;
+    if (layer < 0 || layer >= d.num_layers || num_seqs < 0 || num_q_heads <= 0 || block_table_width <= 0 ||
+        max_context_len < 0 || num_seqs > 65535)
+        return PKV_ERR_ARG;
+    if (num_q_heads % d.num_kv_heads) return PKV_ERR_SHAPE;
+    const int G = num_q_heads / d.num_kv_heads;
+    if (G > 16) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !block_tables || !context_lens || !out) return PKV_ERR_NULL;
+    if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_DTYPE;
+    if (!is_quantized(d.kv_dtype) && q_dtype != d.kv_dtype) return PKV_ERR_DTYPE;
+    if ((reinterpret_cast<uintptr_t>(q) & 3) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
+    int engine = opts ? opts->engine : 0;
+    if (engine < 0 || engine > 2) return PKV_ERR_ARG;
+    if (engine == 0) engine = 1;
+    int P, parts;
+    int rc = decode_partitioning(pool, num_seqs, max_context_len, opts, &P, &parts);
+    if (rc != PKV_OK) return rc;
+    const size_t need = parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (d.head_dim + 2) * sizeof(float) : 0;
+    if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15)))
+        return PKV_ERR_WORKSPACE;
+    const CUtensorMap *tmk = nullptr, *tmv = nullptr;
+    rc = layer_maps(pool, layer, &tmk, &tmv);
+    if (rc != PKV_OK) return rc;
+
+    DecodeArgs a;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.tables = block_tables;
+    a.W = block_table_width;
+    a.ctx_lens = context_lens;
+    a.B = num_seqs;
+    a.H_q = num_q_heads;
+    a.H_kv = d.num_kv_heads;
+    a.G = G;
+    a.N = d.num_blocks;
+    a.d = d.head_dim;
+    a.kv_dtype = d.kv_dtype;
+    a.part_tokens = P;
+    a.max_parts = parts;
+    a.scale = scale;
+    a.k_scale = d.k_scale ? d.k_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.v_scale = d.v_scale ? d.v_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.out = out;
+    float* ws = static_cast<float*>(workspace);
+    a.ws_o = need ? ws : nullptr;
+    a.ws_ml = need ? ws + (size_t)num_seqs * num_q_heads * parts * d.head_dim : nullptr;
+    a.status = d.device_status;
+    a.engine = engine;
+    return launch_decode(a, tmk, tmv, static_cast<cudaStream_t>(stream));
+}
+
+size_t paged_prefill_workspace_bytes(pkv_pool_t pool, int chunk_len, int num_q_heads, int ctx_before)
+{
+    (void)pool;
+    (void)chunk_len;
+    (void)num_q_heads;
+    (void)ctx_before;
+    return 0;
+}
+
+int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, const int32_t* block_table,
+                             int block_table_width, int ctx_before, int chunk_len, int num_q_heads, float scale,
+                             float* out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (!pool) return PKV_ERR_NULL;
+    const pkv_pool_desc& d = pool->d;
+    if (layer < 0 || layer >= d.num_layers || ctx_before < 0 || chunk_len < 0 || num_q_heads <= 0 ||
+        block_table_width <= 0)
+        return PKV_ERR_ARG;
+    if (num_q_heads % d.num_kv_heads) return PKV_ERR_SHAPE;
+    if (is_quantized(d.kv_dtype)) return PKV_ERR_UNSUPPORTED;
+    if (q_dtype != d.kv_dtype) return PKV_ERR_DTYPE;
+    if ((long long)block_table_width * PKV_BLOCK_SIZE < (long long)ctx_before + chunk_len) return PKV_ERR_SHAPE;
+    if (chunk_len == 0) return PKV_OK;
+    if (!q || !block_table || !out) return PKV_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
+    const CUtensorMap *tmk = nullptr, *tmv = nullptr;
+    int rc = layer_maps(pool, layer, &tmk, &tmv);
+    if (rc != PKV_OK) return rc;
+    PrefillArgs a;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.table = block_table;
+    a.W = block_table_width;
+    a.P0 = ctx_before;
+    a.C = chunk_len;
+    a.H_q = num_q_heads;
+    a.H_kv = d.num_kv_heads;
+    a.G = num_q_heads / d.num_kv_heads;
+    a.N = d.num_blocks;
+    a.d = d.head_dim;
+    a.kv_dtype = d.kv_dtype;
+    a.scale = scale;
+    a.out = out;
+    a.status = d.device_status;
+    return launch_prefill(a, tmk, tmv, static_cast<cudaStream_t>(stream));
+}
+
+int pkv_read_device_status(pkv_pool_t pool, void* stream, int32_t* status_out)
+{
+    if (!pool || !status_out) return PKV_ERR_NULL;
+    *status_out = 0;
+    if (!pool->d.device_status) return PKV_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t host = 0;
+    if (cudaMemcpyAsync(&host, pool->d.device_status, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PKV_ERR_CUDA;
+    if (host != 0 && cudaMemsetAsync(pool->d.device_status, 0, sizeof(int32_t), s) != cudaSuccess) return PKV_ERR_CUDA;
+    *status_out = host;
+    if (host & PKV_DEV_TIMEOUT) return PKV_ERR_TIMEOUT;
+    return host ? PKV_ERR_INDEX : PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,459 @@
+// decode.cu -- paged_decode_attn: one query token per sequence against its paged cache.
+//
+// What is computed ("KV cache, continuous batching and paged attention", section "Paged
+// attention": the attention kernel follows the block table; "KV cache, GQA, paging and
+// continuous batching", section "Mechanics": G query heads share one KV head):
+//   out[b][h] = softmax_t(scale * q[b][h] . K_b[t]) V_b[t],  t < context_lens[b],
+// K_b[t] = tile (block_tables[b][t / 16], h / G), row t % 16.
+//
+// Design (B200):
+//   * One warp per (partition of <= part_tokens tokens, KV head, sequence).  The warp
+//     streams its partition's (block, KV head) tiles -- 16 rows of K and of V, each tile
+//     contiguous in HBM -- into a ring of shared-memory stages with tiled TMA loads
+//     (128-byte swizzle, completion on an mbarrier; no multicast).  Lane 0 keeps STAGES
+//     tiles in flight; the block-table slice is read once into shared memory.
+//   * All G query heads of the KV group are processed together, so each K/V byte is
+//     read from HBM exactly once.  Q.K^T and P.V are small dense contractions
+//     (G x d times d x 16 tokens); they run on the tensor cores with warp-level
+//     mma.sync m16n8k16 (fp32 accumulate), which keeps the FP32 pipe free: at G = 8 the
+//     CUDA-core form needs 8 flop per K/V byte, as much as the FP32 pipe can issue at
+//     HBM speed.  Scores: S[16 heads][16 tokens] = Q . K^T with K from ldmatrix;
+//     output: O^T[d][heads] += V^T . P^T with V from ldmatrix.trans.  P is split into a
+//     high and a low 16-bit part (two MMAs) so the P.V product keeps ~16 mantissa bits.
+//   * Online softmax in fp32 in the log2 domain (ex2 on the SFU), row maxima by quad
+//     shuffles.  Masked (past-the-end) tokens get -inf scores and zeroed V, so stale or
+//     poisoned slots never reach the result.
+//   * Split-K: a sequence longer than one partition writes per-partition (o, m, l)
+//     partials; decode_reduce merges them with the log-sum-exp rule.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+constexpr int kMaxPartTiles = 256;   // partition_tokens <= 4096
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeParams {
+    const void* q;
+    const int32_t* tables;
+    const int32_t* ctx_lens;
+    const float* k_scale;
+    const float* v_scale;
+    float* out;
+    float* ws_o;
+    float* ws_ml;
+    int32_t* status;
+    int W, H_q, H_kv, G, N, part_tokens, max_parts;
+    float scale_log2;
+};
+
+// Context length of sequence b, clamped to what the table and the grid can cover.
+__device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool report)
+{
+    int ctx = p.ctx_lens[b];
+    const int cap = min(p.W * kBlock, p.max_parts * p.part_tokens);
+    if (ctx < 0 || ctx > cap) {
+        if (report) flag_status(p.status, PKV_DEV_BAD_LENGTH);
+        ctx = ctx < 0 ? 0 : cap;
+    }
+    return ctx;
+}
+
+// Byte address of 16-byte chunk `c` of row `t` in a tile stored as 128-byte-wide TMA
+// boxes of 16 rows with the 128-byte swizzle (chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t swz128(uint32_t tile, int t, int c)
+{
+    return tile + (uint32_t)((c >> 3) * (16 * 128) + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core engine, 16-bit pools.
+// ---------------------------------------------------------------------------
+template <int D, int STAGES>
+struct Mma16Cfg {
+    static constexpr int TILE = 16 * 2 * D;        // bytes of one K (or V) tile
+    static constexpr int NBOX = D / 64;            // 128-byte boxes per row
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+};
+
+template <int D, bool BF16, int NHT, int STAGES>
+__global__ void __launch_bounds__(32)
+decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV)
+{
+    using Cfg = Mma16Cfg<D, STAGES>;
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ __align__(8) uint64_t bars[STAGES];
+    __shared__ int tbl[kMaxPartTiles];
+
+    const int lane = threadIdx.x;
+    const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int r = lane >> 2, qd = lane & 3;
+    const int hbase = g * p.G;
+
+    const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
+    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
+    const int tok0 = part * p.part_tokens;
+    if (tok0 >= ctx) {
+        if (part == 0) {   // empty context: a zero row
+            float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
+            for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
+        }
+        return;
+    }
+    const int ntok = min(p.part_tokens, ctx - tok0);
+    const int ntiles = (ntok + kBlock - 1) / kBlock;
+
+    const int32_t* trow = p.tables + (size_t)b * p.W + tok0 / kBlock;
+    for (int j = lane; j < ntiles; j += 32) {
+        int blk = trow[j];
+        if ((unsigned)blk >= (unsigned)p.N) {
+            flag_status(p.status, PKV_DEV_BAD_BLOCK);
+            blk = 0;
+        }
+        tbl[j] = blk;
+    }
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    if (lane == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        mbar_fence_init();
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    __syncwarp();
+
+    auto issue = [&](int j) {
+        const int s = j % STAGES;
+        const uint32_t bar = smem_u32(&bars[s]);
+        const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
+        const int row = (tbl[j] * p.H_kv + g) * kBlock;
+        mbar_arrive_expect_tx(bar, Cfg::STAGE);
+#pragma unroll
+        for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + x * 2048, &tmK, x * 64, row, bar);
+#pragma unroll
+        for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + Cfg::TILE + x * 2048, &tmV, x * 64, row, bar);
+    };
+    if (lane == 0) {
+        for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
+    }
+
+    // Q as the A operand of S = Q.K^T: rows = heads (r and r + 8), 16 dims per k-step.
+    uint32_t qa[D / 16][4];
+    {
+        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(
+            static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D);
+        const bool r0 = r < p.G, r1 = (NHT == 2) && (r + 8 < p.G);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            qa[ks][0] = r0 ? __ldg(q32 + (r * D + 16 * ks + 2 * qd) / 2) : 0u;
+            qa[ks][2] = r0 ? __ldg(q32 + (r * D + 16 * ks + 8 + 2 * qd) / 2) : 0u;
+            qa[ks][1] = r1 ? __ldg(q32 + ((r + 8) * D + 16 * ks + 2 * qd) / 2) : 0u;
+            qa[ks][3] = r1 ? __ldg(q32 + ((r + 8) * D + 16 * ks + 8 + 2 * qd) / 2) : 0u;
+        }
+    }
+
+    float o[D / 16][NHT][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+        for (int hn = 0; hn < NHT; ++hn)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[mt][hn][c] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    const float sl = p.scale_log2;
+
+    int j = 0;
+    bool ok = true;
+    for (; j < ntiles; ++j) {
+        const int s = j % STAGES;
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1)) {
+            ok = false;
+            break;
+        }
+        const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
+        const uint32_t vb = kb + Cfg::TILE;
+        const int nv = min(kBlock, ntok - j * kBlock);
+
+        // S = Q . K^T  (two n-tiles of 8 tokens)
+        float sc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bk[4];
+                ldsm_x4(bk, swz128(kb, nt * 8 + (lane & 7), 4 * kk + (lane >> 3)));
+                mma16816<BF16>(sc[nt], qa[2 * kk], bk[0], bk[1]);
+                mma16816<BF16>(sc[nt], qa[2 * kk + 1], bk[2], bk[3]);
+            }
+        }
+
+        // online softmax, rows r (c = 0, 1) and r + 8 (c = 2, 3)
+        float pr[2][4];
+        float alpha[2];
+#pragma unroll
+        for (int hr = 0; hr < NHT; ++hr) {
+            float x[2][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = nt * 8 + 2 * qd + e;
+                    x[nt][e] = tok < nv ? sc[nt][2 * hr + e] * sl : -INFINITY;
+                    mx = fmaxf(mx, x[nt][e]);
+                }
+            mx = warp_max_quad(mx);
+            const float mn = fmaxf(m_run[hr], mx);   // finite: every tile has a valid token
+            alpha[hr] = ex2(m_run[hr] - mn);
+            float sum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    pr[nt][2 * hr + e] = ex2(x[nt][e] - mn);
+                    sum += pr[nt][2 * hr + e];
+                }
+            l_run[hr] = l_run[hr] * alpha[hr] + sum;
+            m_run[hr] = mn;
+        }
+
+        // rescale O^T columns (heads 2qd, 2qd + 1 of each head n-tile) when a max moved
+        const bool moved = (alpha[0] != 1.f) || (NHT == 2 && alpha[1] != 1.f);
+        if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+            for (int hn = 0; hn < NHT; ++hn) {
+                const float a_lo = __shfl_sync(0xffffffffu, alpha[hn], 8 * qd);
+                const float a_hi = __shfl_sync(0xffffffffu, alpha[hn], 8 * qd + 4);
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    o[mt][hn][0] *= a_lo;
+                    o[mt][hn][1] *= a_hi;
+                    o[mt][hn][2] *= a_lo;
+                    o[mt][hn][3] *= a_hi;
+                }
+            }
+        }
+
+        // P^T as the B operand of O^T += V^T . P^T (k = tokens, n = heads), hi + lo parts
+        uint32_t bh[NHT][2], bl[NHT][2];
+#pragma unroll
+        for (int hn = 0; hn < NHT; ++hn)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float p0 = pr[nt][2 * hn], p1 = pr[nt][2 * hn + 1];
+                bh[hn][nt] = pack2<BF16>(p0, p1);
+                const float2 back = unpack2<BF16>(bh[hn][nt]);
+                bl[hn][nt] = pack2<BF16>(p0 - back.x, p1 - back.y);
+            }
+
+        uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
+        if (nv < kBlock) {   // zero V of past-the-end tokens (their P is 0, their V may be stale)
+            keep01 = (2 * qd < nv ? 0x0000ffffu : 0u) | (2 * qd + 1 < nv ? 0xffff0000u : 0u);
+            keep23 = (8 + 2 * qd < nv ? 0x0000ffffu : 0u) | (9 + 2 * qd < nv ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            uint32_t va[4];
+            ldsm_x4_trans(va, swz128(vb, ((lane >> 4) << 3) + (lane & 7), 2 * mt + ((lane >> 3) & 1)));
+            va[0] &= keep01;
+            va[1] &= keep01;
+            va[2] &= keep23;
+            va[3] &= keep23;
+#pragma unroll
+            for (int hn = 0; hn < NHT; ++hn) {
+                mma16816<BF16>(o[mt][hn], va, bh[hn][0], bh[hn][1]);
+                mma16816<BF16>(o[mt][hn], va, bl[hn][0], bl[hn][1]);
+            }
+        }
+
+        __syncwarp();
+        if (lane == 0 && j + STAGES < ntiles) {
+            fence_proxy_async_smem();
+            issue(j + STAGES);
+        }
+    }
+
+    if (!ok) {
+        if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
+        for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
+            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
+        return;
+    }
+
+    // ---- epilogue: O rows [head][dim] through shared memory, then coalesced stores
+#pragma unroll
+    for (int hr = 0; hr < NHT; ++hr) l_run[hr] = warp_sum_quad(l_run[hr]);
+    const bool final_out = (nparts == 1);
+    float* so = reinterpret_cast<float*>(smem);
+    constexpr int SR = D + 4;   // padded row stride (floats)
+    __syncwarp();
+#pragma unroll
+    for (int hn = 0; hn < NHT; ++hn) {
+        float inv_lo = 1.f, inv_hi = 1.f;
+        const float la = __shfl_sync(0xffffffffu, l_run[hn], 8 * qd);
+        const float lb = __shfl_sync(0xffffffffu, l_run[hn], 8 * qd + 4);
+        if (final_out) {
+            inv_lo = 1.f / la;
+            inv_hi = 1.f / lb;
+        }
+        const int h0 = 8 * hn + 2 * qd;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            so[h0 * SR + 16 * mt + r] = o[mt][hn][0] * inv_lo;
+            so[(h0 + 1) * SR + 16 * mt + r] = o[mt][hn][1] * inv_hi;
+            so[h0 * SR + 16 * mt + 8 + r] = o[mt][hn][2] * inv_lo;
+            so[(h0 + 1) * SR + 16 * mt + 8 + r] = o[mt][hn][3] * inv_hi;
+        }
+    }
+    __syncwarp();
+    const size_t row0 = (size_t)b * p.H_q + hbase;
+    if (final_out) {
+        for (int i = lane; i < p.G * (D / 4); i += 32) {
+            const int h = i / (D / 4), c4 = i % (D / 4);
+            const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
+            *reinterpret_cast<float4*>(p.out + (row0 + h) * D + 4 * c4) = v;
+        }
+    } else {
+        for (int i = lane; i < p.G * (D / 4); i += 32) {
+            const int h = i / (D / 4), c4 = i % (D / 4);
+            const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
+            *reinterpret_cast<float4*>(p.ws_o + ((row0 + h) * p.max_parts + part) * D + 4 * c4) = v;
+        }
+        if (qd == 0) {
+#pragma unroll
+            for (int hr = 0; hr < NHT; ++hr) {
+                const int h = r + 8 * hr;
+                if (h < p.G) {
+                    float2 ml = make_float2(m_run[hr], l_run[hr]);
+                    *reinterpret_cast<float2*>(p.ws_ml + ((row0 + h) * p.max_parts + part) * 2) = ml;
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-K merge: out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
+// One warp per (query head, sequence); sequences that fit one partition were written
+// directly by the main kernel and are skipped.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
+{
+    const int h = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
+    const int ctx = checked_ctx(p, b, false);
+    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
+    if (nparts <= 1) return;
+    const size_t base = ((size_t)b * p.H_q + h) * p.max_parts;
+    const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + base;
+    float M = -INFINITY;
+    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int i = lane; i < nparts; i += 32) L += ex2(ml[i].x - M) * ml[i].y;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+
+    constexpr int V = D / 32;   // floats per lane
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    const float* po = p.ws_o + base * D + lane * V;
+#pragma unroll 4
+    for (int i = 0; i < nparts; ++i) {
+        const float w = ex2(ml[i].x - M);
+        if constexpr (V == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(po + (size_t)i * D);
+            acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2*>(po + (size_t)i * D);
+            acc[0] += w * v.x; acc[1] += w * v.y;
+        }
+    }
+    const float inv = 1.f / L;
+    float* out = p.out + ((size_t)b * p.H_q + h) * D + lane * V;
+    if constexpr (V == 4) {
+        *reinterpret_cast<float4*>(out) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else {
+        *reinterpret_cast<float2*>(out) = make_float2(acc[0] * inv, acc[1] * inv);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launcher
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kStages = 4;
+
+template <typename K>
+int launch_k(K kernel, int smem, dim3 grid, cudaStream_t s, const DecodeParams& p, const CUtensorMap* tmk,
+             const CUtensorMap* tmv)
+{
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    kernel<<<grid, 32, smem, s>>>(p, *tmk, *tmv);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+int launch_mma16(const DecodeParams& p, int nht, dim3 grid, cudaStream_t s, const CUtensorMap* tmk,
+                 const CUtensorMap* tmv)
+{
+    constexpr int smem = Mma16Cfg<D, kStages>::SMEM;
+    if (nht == 1) return launch_k(decode_mma16_kernel<D, BF16, 1, kStages>, smem, grid, s, p, tmk, tmv);
+    return launch_k(decode_mma16_kernel<D, BF16, 2, kStages>, smem, grid, s, p, tmk, tmv);
+}
+
+}  // namespace
+
+int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s)
+{
+    DecodeParams p;
+    p.q = a.q;
+    p.tables = a.tables;
+    p.ctx_lens = a.ctx_lens;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.out = a.out;
+    p.ws_o = a.ws_o;
+    p.ws_ml = a.ws_ml;
+    p.status = a.status;
+    p.W = a.W;
+    p.H_q = a.H_q;
+    p.H_kv = a.H_kv;
+    p.G = a.G;
+    p.N = a.N;
+    p.part_tokens = a.part_tokens;
+    p.max_parts = a.max_parts;
+    p.scale_log2 = a.scale * kLog2e;
+
+    const dim3 grid(a.max_parts, a.H_kv, a.B);
+    const int nht = a.G <= 8 ? 1 : 2;
+    int rc = PKV_ERR_UNSUPPORTED;
+    if (a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) {
+        if (a.engine != 1) return PKV_ERR_UNSUPPORTED;
+        const bool bf = a.kv_dtype == PKV_BF16;
+        if (a.d == 128) rc = bf ? launch_mma16<128, true>(p, nht, grid, s, tmk, tmv)
+                                : launch_mma16<128, false>(p, nht, grid, s, tmk, tmv);
+        else if (a.d == 64) rc = bf ? launch_mma16<64, true>(p, nht, grid, s, tmk, tmv)
+                                    : launch_mma16<64, false>(p, nht, grid, s, tmk, tmv);
+    }
+    if (rc != PKV_OK) return rc;
+    if (a.max_parts > 1) {
+        const dim3 rgrid(a.H_q, a.B);
+        if (a.d == 128) decode_reduce_kernel<128><<<rgrid, 32, 0, s>>>(p);
+        else decode_reduce_kernel<64><<<rgrid, 32, 0, s>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
+
+}  // namespace pkv

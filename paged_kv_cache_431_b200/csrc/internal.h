@@ -1,0 +1,83 @@
+// internal.h -- host-side types shared by the C-ABI implementation and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/pkv.h"
+
+struct pkv_pool {
+    pkv_pool_desc d;
+    int row_bytes;             // bytes of one token row of one KV head
+    size_t tile_bytes;         // 16 rows: one (block, kv head) tile
+    size_t layer_bytes;        // bytes of one layer's K (or V) pool
+    size_t layer_scales;       // fp32 scales per layer (N * H_kv), 0 for 16-bit pools
+    std::mutex mu;             // guards the lazily built tensor maps
+    bool maps_ready = false;
+    std::vector<CUtensorMap> tmk, tmv;   // per layer: K and V pool as a 2-D tensor
+};
+
+namespace pkv {
+
+int row_bytes_of(int dtype, int head_dim);
+bool is_quantized(int dtype);
+
+// Tensor maps for `layer` (built on first use). Returns PKV_OK or PKV_ERR_CUDA.
+int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtensorMap** tmv);
+
+int num_sms();
+
+struct DecodeArgs {
+    const void* q;
+    int q_dtype;
+    const int32_t* tables;
+    int W;
+    const int32_t* ctx_lens;
+    int B, H_q, H_kv, G, N, d;
+    int kv_dtype;
+    int part_tokens, max_parts;
+    float scale;
+    const float* k_scale;   // this layer's scales, or null
+    const float* v_scale;
+    float* out;
+    float* ws_o;            // [B][H_q][max_parts][d]
+    float* ws_ml;           // [B][H_q][max_parts][2]
+    int32_t* status;
+    int engine;             // 1 mma, 2 fma
+};
+
+int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
+
+struct AppendArgs {
+    const void* k;
+    const void* v;
+    const int32_t* slots;
+    int T, N, H_kv, d, kv_dtype;
+    uint8_t* k_pool;        // this layer
+    uint8_t* v_pool;
+    float* k_scale;         // this layer, quantized only
+    float* v_scale;
+    void* workspace;        // quantized only: per-block scratch
+    int32_t* status;
+};
+
+int launch_append(const AppendArgs& a, cudaStream_t s);
+size_t append_workspace_bytes(int N, int H_kv, int kv_dtype);
+
+struct PrefillArgs {
+    const void* q;
+    int q_dtype;
+    const int32_t* table;
+    int W, P0, C, H_q, H_kv, G, N, d;
+    int kv_dtype;
+    float scale;
+    float* out;
+    int32_t* status;
+};
+
+int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
+
+}  // namespace pkv

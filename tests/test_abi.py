@@ -1,0 +1,123 @@
+"""CPU checks of the C-ABI boundary: the library loads without a GPU, exports every
+entry point include/pkv.h declares, sizes pools by the memory equation, and rejects bad
+arguments on the host (no CUDA call is reached by these cases)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from paged_kv_cache_431_b200 import pkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    return re.findall(r"^PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, re.M)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_functions())
+    for n in ("kv_pool_create", "kv_append", "paged_decode_attn", "paged_prefill_chunk_attn"):
+        assert n in names
+    assert len(names) >= 12
+
+
+def test_library_exports_every_declared_symbol():
+    L = pkv.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert L.pkv_version() >= 100
+    assert pkv.strerror(0) == "ok" and "workspace" in pkv.strerror(-5)
+
+
+@pytest.mark.parametrize("dtype,nbytes", [(pkv.BF16, 2), (pkv.F16, 2), (pkv.INT8, 1), (pkv.FP8E4M3, 1)])
+def test_pool_bytes_follow_the_memory_equation(dtype, nbytes):
+    """K + V pool bytes for N blocks == the oracle's cache size for N * 16 tokens."""
+    for (L, N, H, d) in ((80, 43520, 8, 128), (1, 64, 2, 64), (1, 131072, 8, 128)):
+        kb, sb = pkv.pkv_pool_bytes(L, N, H, d, dtype)
+        assert 2 * kb == oracle.kv_cache_bytes(L, H, d, nbytes, N * 16, 1)
+        assert sb == (L * N * H * 4 if dtype in pkv.QUANTIZED else 0)
+
+
+def test_int4_pool_bytes_are_half_of_int8():
+    kb8, _ = pkv.pkv_pool_bytes(1, 1000, 8, 128, pkv.INT8)
+    kb4, _ = pkv.pkv_pool_bytes(1, 1000, 8, 128, pkv.INT4)
+    assert kb4 * 2 == kb8
+
+
+def _desc(**kw):
+    base = dict(num_layers=1, num_blocks=64, block_size=16, num_kv_heads=2, head_dim=64, kv_dtype=pkv.F16,
+                k_data=0x10000, v_data=0x20000, k_scale=None, v_scale=None, device_status=None)
+    base.update(kw)
+    return pkv._PoolDesc(*[base[f] for f, _ in pkv._PoolDesc._fields_])
+
+
+def _create(**kw):
+    h = ctypes.c_void_p()
+    rc = pkv.lib().kv_pool_create(ctypes.byref(_desc(**kw)), ctypes.byref(h))
+    return rc, h
+
+
+def test_pool_create_validation():
+    L = pkv.lib()
+    rc, h = _create()
+    assert rc == 0 and h.value
+    assert L.kv_pool_destroy(h) == 0
+    assert L.kv_pool_destroy(None) == 0
+    assert L.kv_pool_create(None, ctypes.byref(ctypes.c_void_p())) == -1
+    assert _create(block_size=8)[0] == -2
+    assert _create(head_dim=96)[0] == -9
+    assert _create(kv_dtype=7)[0] == -3
+    assert _create(k_data=None)[0] == -1
+    assert _create(k_data=0x10008)[0] == -2              # not 16-byte aligned
+    assert _create(kv_dtype=pkv.INT8)[0] == -1           # quantized without scales
+    assert _create(kv_dtype=pkv.INT8, k_scale=0x30000, v_scale=0x40000)[0] == 0
+    assert _create(num_blocks=0)[0] == -2
+
+
+def test_decode_and_append_argument_checks():
+    L = pkv.lib()
+    rc, h = _create(num_kv_heads=2, head_dim=64)
+    assert rc == 0
+    P = ctypes.c_void_p
+    fake = P(0x50000)
+    try:
+        # H_q not a multiple of H_kv
+        assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 3, 64, 0.1, fake, None, 0, None, None) == -4
+        # G = 20 > 16
+        assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 40, 64, 0.1, fake, None, 0, None, None) == -9
+        # q dtype must match a 16-bit pool
+        assert L.paged_decode_attn(h, 0, fake, pkv.BF16, fake, 4, fake, 4, 8, 64, 0.1, fake, None, 0, None, None) == -3
+        # bad layer
+        assert L.paged_decode_attn(h, 1, fake, pkv.F16, fake, 4, fake, 4, 8, 64, 0.1, fake, None, 0, None, None) == -2
+        # a split-K grid needs a workspace
+        assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 8, 100000, 0.1, fake, None, 0, None,
+                                   None) == -5
+        # empty batch is a no-op
+        assert L.paged_decode_attn(h, 0, None, pkv.F16, None, 4, None, 0, 8, 0, 0.1, None, None, 0, None, None) == 0
+        # append: source dtype must equal a 16-bit pool's dtype; zero tokens is a no-op
+        assert L.kv_append(h, 0, fake, fake, pkv.BF16, fake, 3, None, 0, None) == -3
+        assert L.kv_append(h, 0, None, None, pkv.F16, None, 0, None, 0, None) == 0
+        # prefill: table too narrow for the chunk
+        assert L.paged_prefill_chunk_attn(h, 0, fake, pkv.F16, fake, 2, 20, 20, 8, 0.1, fake, None, 0, None) == -4
+        assert L.paged_decode_workspace_bytes(h, 4, 8, 64, None) == 0          # one partition
+        assert L.paged_decode_workspace_bytes(h, 4, 8, 4096, None) > 0
+    finally:
+        L.kv_pool_destroy(h)
+
+
+def test_quantized_append_needs_bf16_source_and_workspace():
+    L = pkv.lib()
+    rc, h = _create(kv_dtype=pkv.INT8, k_scale=0x30000, v_scale=0x40000)
+    fake = ctypes.c_void_p(0x50000)
+    try:
+        need = L.kv_append_workspace_bytes(h, 10)
+        assert need == (2 * 64 * 2 + 64) * 4
+        assert L.kv_append(h, 0, fake, fake, pkv.F16, fake, 10, fake, need, None) == -3
+        assert L.kv_append(h, 0, fake, fake, pkv.BF16, fake, 10, None, 0, None) == -5
+        assert L.kv_append(h, 0, fake, fake, pkv.BF16, fake, 10, fake, need - 4, None) == -5
+    finally:
+        L.kv_pool_destroy(h)
