@@ -196,3 +196,22 @@ def kv_source(T: int, H_kv: int, d: int, gen: torch.Generator, device="cpu",
         k.view(T, H_kv * d)[:, idx] *= outlier_gain
         v.view(T, H_kv * d)[:, idx] *= outlier_gain
     return k, v
+
+
+def compact_subset(tables: torch.Tensor, ctx_lens: torch.Tensor, seq_ids):
+    """For sequences `seq_ids`: the physical blocks they reference (sorted) and their
+    tables renumbered into that list."""
+    seq_ids = list(seq_ids)
+    sub_t = tables[seq_ids].clone()
+    sub_c = ctx_lens[seq_ids].clone()
+    used = []
+    for r, b in enumerate(seq_ids):
+        nb = ceil_div(int(ctx_lens[b]), BLOCK)
+        used.extend(int(x) for x in tables[b, :nb])
+    uniq = sorted(set(used))
+    remap = {blk: i for i, blk in enumerate(uniq)}
+    for r, b in enumerate(seq_ids):
+        nb = ceil_div(int(ctx_lens[b]), BLOCK)
+        for j in range(nb):
+            sub_t[r, j] = remap[int(tables[b, j])]
+    return uniq, sub_t, sub_c

@@ -9,6 +9,7 @@ import torch
 
 import oracle
 from paged_kv_cache_431_b200 import workloads as wl
+from paged_kv_cache_431_b200.workloads import compact_subset  # noqa: F401
 
 TOL = 2e-3   # max |GPU - oracle| for fp32 attention outputs
 
@@ -27,25 +28,6 @@ def oracle_pool_from_tensors(k_pool, v_pool, dtype, k_scale=None, v_scale=None) 
     ks = None if k_scale is None else k_scale.detach().cpu().numpy()
     vs = None if v_scale is None else v_scale.detach().cpu().numpy()
     return oracle.Pool(N, H, d, dtype, raw(k_pool), raw(v_pool), ks, vs)
-
-
-def compact_subset(tables: torch.Tensor, ctx_lens: torch.Tensor, seq_ids):
-    """For sequences `seq_ids`: the physical blocks they reference (sorted) and their
-    tables renumbered into that list."""
-    seq_ids = list(seq_ids)
-    sub_t = tables[seq_ids].clone()
-    sub_c = ctx_lens[seq_ids].clone()
-    used = []
-    for r, b in enumerate(seq_ids):
-        nb = wl.ceil_div(int(ctx_lens[b]), wl.BLOCK)
-        used.extend(int(x) for x in tables[b, :nb])
-    uniq = sorted(set(used))
-    remap = {blk: i for i, blk in enumerate(uniq)}
-    for r, b in enumerate(seq_ids):
-        nb = wl.ceil_div(int(ctx_lens[b]), wl.BLOCK)
-        for j in range(nb):
-            sub_t[r, j] = remap[int(tables[b, j])]
-    return uniq, sub_t, sub_c
 
 
 def oracle_subset_pool(k_pool, v_pool, dtype, blocks, k_scale=None, v_scale=None) -> oracle.Pool:
