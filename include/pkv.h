@@ -180,6 +180,32 @@ PKV_API int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_d
                       void* workspace, size_t workspace_bytes,
                       const pkv_decode_opts* opts, void* stream);
 
+/* Size of the fixed device buffer paged_decode_attn_noalloc keeps its split-K partials in. */
+#define PKV_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * paged_decode_attn_noalloc -- paged_decode_attn for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call; it exists for callers embedded in a
+ * host runtime that owns every device allocation (a serving engine's memory planner, a
+ * plugin that may only touch the memory it is given) and for latency-critical paths where
+ * a cudaMalloc, which may synchronize the device, is not acceptable.
+ * Same arguments, result and errors as paged_decode_attn, minus the workspace: the split-K
+ * partials go to a buffer of PKV_NOALLOC_SCRATCH_BYTES (32 MiB) that the library holds in
+ * device memory on every GPU that loads it, until the process exits.  A call whose
+ * partials (paged_decode_workspace_bytes for the same sizes and options) exceed that size
+ * returns PKV_ERR_WORKSPACE without launching anything.  The call allocates nothing.
+ * The first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture on the device.
+ * All calls share the buffer and it keeps the last call's contents (no call relies on them:
+ * each writes every partial it reads).  Calls whose kernels may overlap on the GPU race on
+ * the buffer; issue them in order on one stream.
+ */
+PKV_API int paged_decode_attn_noalloc(pkv_pool_t pool, int layer, const void* q, int q_dtype,
+                                      const int32_t* block_tables, int block_table_width,
+                                      const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                      int max_context_len, float scale, float* out,
+                                      const pkv_decode_opts* opts, void* stream);
+
 /* Workspace paged_prefill_chunk_attn needs (bytes). */
 PKV_API size_t paged_prefill_workspace_bytes(pkv_pool_t pool, int chunk_len, int num_q_heads, int ctx_before);
 

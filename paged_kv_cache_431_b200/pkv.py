@@ -234,6 +234,31 @@ def paged_decode_attn(pool: KVPool, layer: int, q: torch.Tensor, block_tables: t
     return out
 
 
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def paged_decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, block_tables: torch.Tensor,
+                              context_lens: torch.Tensor, scale: float, max_context_len: int,
+                              out: torch.Tensor | None = None, engine: int = 0, partition_tokens: int = 0,
+                              stream=None) -> torch.Tensor:
+    """paged_decode_attn without a workspace argument, for callers that cannot allocate device
+    memory for one: the split-K partials use the library's fixed 32 MiB device buffer.  Only
+    the output is the caller's.  Calls that may overlap on the GPU share that buffer and race;
+    issue them in order on one stream."""
+    L = lib()
+    fn = L.paged_decode_attn_noalloc
+    P, i32 = ctypes.c_void_p, ctypes.c_int
+    fn.restype = i32
+    fn.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, ctypes.c_float, P, P, P]
+    B, H_q, d = q.shape
+    if out is None:
+        out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
+    _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_tables), block_tables.shape[1],
+              _ptr(context_lens), B, H_q, max_context_len, float(scale), _ptr(out),
+              _opts(engine, partition_tokens), _stream(stream)), "paged_decode_attn_noalloc")
+    return out
+
+
 def paged_prefill_chunk_attn(pool: KVPool, layer: int, q: torch.Tensor, block_table: torch.Tensor,
                              ctx_before: int, scale: float, out: torch.Tensor | None = None,
                              stream=None) -> torch.Tensor:
