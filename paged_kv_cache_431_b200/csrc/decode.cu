@@ -25,46 +25,9 @@
 //     poisoned slots never reach the result.
 //   * Split-K: a sequence longer than one partition writes per-partition (o, m, l)
 //     partials; decode_reduce merges them with the log-sum-exp rule.
-#include "common.cuh"
-#include "internal.h"
+#include "decode_common.cuh"
 
 namespace pkv {
-
-constexpr int kMaxPartTiles = 256;   // partition_tokens <= 4096
-constexpr float kLog2e = 1.4426950408889634f;
-
-struct DecodeParams {
-    const void* q;
-    const int32_t* tables;
-    const int32_t* ctx_lens;
-    const float* k_scale;
-    const float* v_scale;
-    float* out;
-    float* ws_o;
-    float* ws_ml;
-    int32_t* status;
-    int W, H_q, H_kv, G, N, part_tokens, max_parts;
-    float scale_log2;
-};
-
-// Context length of sequence b, clamped to what the table and the grid can cover.
-__device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool report)
-{
-    int ctx = p.ctx_lens[b];
-    const int cap = min(p.W * kBlock, p.max_parts * p.part_tokens);
-    if (ctx < 0 || ctx > cap) {
-        if (report) flag_status(p.status, PKV_DEV_BAD_LENGTH);
-        ctx = ctx < 0 ? 0 : cap;
-    }
-    return ctx;
-}
-
-// Byte address of 16-byte chunk `c` of row `t` in a tile stored as 128-byte-wide TMA
-// boxes of 16 rows with the 128-byte swizzle (chunk index XOR row % 8).
-__device__ __forceinline__ uint32_t swz128(uint32_t tile, int t, int c)
-{
-    return tile + (uint32_t)((c >> 3) * (16 * 128) + t * 128 + (((c & 7) ^ (t & 7)) << 4));
-}
 
 // ---------------------------------------------------------------------------
 // Tensor-core engine, 16-bit pools.
@@ -433,6 +396,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.N = a.N;
     p.part_tokens = a.part_tokens;
     p.max_parts = a.max_parts;
+    p.q_bf16 = a.q_dtype == PKV_BF16;
     p.scale_log2 = a.scale * kLog2e;
 
     const dim3 grid(a.max_parts, a.H_kv, a.B);
@@ -445,6 +409,9 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
                                 : launch_mma16<128, false>(p, nht, grid, s, tmk, tmv);
         else if (a.d == 64) rc = bf ? launch_mma16<64, true>(p, nht, grid, s, tmk, tmv)
                                     : launch_mma16<64, false>(p, nht, grid, s, tmk, tmv);
+    } else if (is_quantized(a.kv_dtype)) {
+        if (a.engine != 1) return PKV_ERR_UNSUPPORTED;
+        rc = launch_decode_quant(p, a.kv_dtype, a.d, nht, grid, s, tmk, tmv);
     }
     if (rc != PKV_OK) return rc;
     if (a.max_parts > 1) {

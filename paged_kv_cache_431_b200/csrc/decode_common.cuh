@@ -1,0 +1,51 @@
+// decode_common.cuh -- pieces shared by the decode kernels (16-bit and quantized pools).
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+constexpr int kMaxPartTiles = 256;   // partition_tokens <= 4096
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecodeParams {
+    const void* q;
+    const int32_t* tables;
+    const int32_t* ctx_lens;
+    const float* k_scale;
+    const float* v_scale;
+    float* out;
+    float* ws_o;
+    float* ws_ml;
+    int32_t* status;
+    int W, H_q, H_kv, G, N, part_tokens, max_parts;
+    int q_bf16;             // q dtype: 1 bf16, 0 f16
+    float scale_log2;
+};
+
+// Context length of sequence b, clamped to what the table and the grid can cover.
+__device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool report)
+{
+    int ctx = p.ctx_lens[b];
+    const int cap = min(p.W * kBlock, p.max_parts * p.part_tokens);
+    if (ctx < 0 || ctx > cap) {
+        if (report) flag_status(p.status, PKV_DEV_BAD_LENGTH);
+        ctx = ctx < 0 ? 0 : cap;
+    }
+    return ctx;
+}
+
+// Byte address of 16-byte chunk `c` of row `t` in a tile stored as 128-byte-wide TMA
+// boxes of 16 rows with the 128-byte swizzle (chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t swz128(uint32_t tile, int t, int c)
+{
+    return tile + (uint32_t)((c >> 3) * (16 * 128) + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
+
+// Launch the quantized-pool decode kernel (decode_quant.cu).
+int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,
+                        const CUtensorMap* tmk, const CUtensorMap* tmv);
+
+}  // namespace pkv

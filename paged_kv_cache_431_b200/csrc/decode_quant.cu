@@ -1,0 +1,485 @@
+// decode_quant.cu -- paged_decode_attn over quantized pools (int8, fp8 e4m3, int4).
+//
+// Inference guide a2-inf-2, section "KV-cache quantization": keys and values stored as
+// 8- or 4-bit codes sharing one scale; "KV cache, continuous batching and paged
+// attention", section "The KV cache": an fp8 or int8 cache.  Here every (block, KV
+// head) tile carries one fp32 scale for K and one for V, and a value is code * scale.
+//
+// Same structure as the 16-bit kernel (one warp per partition x KV head x sequence,
+// TMA ring of K/V code tiles, online softmax, split-K partials), with dequantization
+// fused into the fragment loads:
+//   * codes are converted to fp16 in registers -- int8 and int4 by the exponent
+//     trick (the code + bias placed in the mantissa of 1024.0, then the bias
+//     subtracted: exact), fp8 e4m3 by the hardware e4m3x2 -> f16x2 conversion
+//     (exact) -- and fed to mma.sync m16n8k16 (f16 in, fp32 accumulate); q is
+//     converted to fp16 once per warp;
+//   * the K scale of a tile multiplies that tile's scores, the V scale multiplies P
+//     before P . V, so the MMAs see plain integer-valued or fp8-valued operands;
+//   * which physical head dims feed which MMA k-slot is chosen so that every lane
+//     reads contiguous code bytes (a dot product does not depend on the order of its
+//     terms); q's fragments use the same assignment.  Output dims are mapped back in
+//     the epilogue.
+#include <cuda_fp8.h>
+
+#include "decode_common.cuh"
+
+namespace pkv {
+
+namespace {
+
+template <int DT, int D>
+struct QCfg {
+    static constexpr int ROW = DT == PKV_INT4 ? D / 2 : D;     // bytes per token row
+    static constexpr int TILE = 16 * ROW;                      // one (block, head) tile
+    static constexpr int STAGE = 2 * TILE;                     // K and V
+    static constexpr int STAGES = DT == PKV_INT4 ? 8 : 6;
+    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static constexpr int SWZ = ROW == 128 ? 7 : ROW == 64 ? 3 : 1;   // TMA 128/64/32-byte swizzle
+    static constexpr int KRUN = ROW / 4;                       // K bytes per lane per token
+    static constexpr int VRUN = ROW / 8;                       // V bytes per lane per row
+    static constexpr int KS = D / 16;                          // MMA k-steps of Q.K^T
+    static constexpr int MT = D / 16;                          // MMA m-tiles of O^T
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+};
+
+// Address of byte `off` (< ROW) of row `t` of a tile written by TMA with the swizzle that
+// XORs the 16-byte chunk index with address bits 7.. of the row start.
+template <int ROW, int SWZ>
+__device__ __forceinline__ uint32_t qaddr(uint32_t tile, int t, int off)
+{
+    const int base = t * ROW;
+    return tile + (uint32_t)(base + ((((off >> 4) ^ ((base >> 7) & SWZ)) << 4) | (off & 15)));
+}
+
+template <int N>
+__device__ __forceinline__ void lds_words(uint32_t (&w)[N], uint32_t addr);
+
+template <>
+__device__ __forceinline__ void lds_words<4>(uint32_t (&w)[4], uint32_t addr)
+{
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_words<2>(uint32_t (&w)[2], uint32_t addr)
+{
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
+}
+template <>
+__device__ __forceinline__ void lds_words<1>(uint32_t (&w)[1], uint32_t addr)
+{
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(addr));
+}
+
+// `bytes` code bytes from row t at byte `off` (16-byte pieces are swizzled separately).
+template <int ROW, int SWZ, int BYTES>
+__device__ __forceinline__ void load_run(uint32_t (&w)[BYTES / 4], uint32_t tile, int t, int off)
+{
+    if constexpr (BYTES >= 16) {
+#pragma unroll
+        for (int c = 0; c < BYTES / 16; ++c) {
+            uint32_t q[4];
+            lds_words<4>(q, qaddr<ROW, SWZ>(tile, t, off + 16 * c));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[4 * c + i] = q[i];
+        }
+    } else {
+        lds_words<BYTES / 4>(w, qaddr<ROW, SWZ>(tile, t, off));
+    }
+}
+
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, float c)
+{
+    __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), __float2half2_rn(c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// int8 codes, already XORed with 0x80 (u = c + 128): two bytes of w chosen by `sel` ->
+// fp16 pair; 0x64XX as fp16 is 1024 + XX.
+__device__ __forceinline__ uint32_t i8x2(uint32_t wx, uint32_t sel)
+{
+    return h2_sub(__byte_perm(wx, 0x64646464u, sel), 1152.f);
+}
+
+// int4 codes, already XORed with 0x8 per nibble (u = c + 8): nibble s of each 16-bit half.
+__device__ __forceinline__ uint32_t i4x2(uint32_t wx, int s)
+{
+    return h2_sub(((wx >> (4 * s)) & 0x000f000fu) | 0x64006400u, 1032.f);
+}
+
+// e4m3 pair (low byte -> low half) -> fp16 pair.
+__device__ __forceinline__ uint32_t e4m3x2(uint32_t w16)
+{
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w16 & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// Physical head dim that feeds MMA k-slot e (0..3: logical 2qd, 2qd+1, 2qd+8, 2qd+9)
+// of k-step ks for lane group qd.
+template <int DT, int D>
+__device__ __forceinline__ int kdim(int ks, int qd, int e)
+{
+    using C = QCfg<DT, D>;
+    if constexpr (DT == PKV_INT4) {
+        const int i = (ks & 1) * 2 + (e >> 1) + (e & 1) * 4;   // nibble of the word
+        return qd * 2 * C::KRUN + 8 * (ks >> 1) + i;
+    } else {
+        return qd * C::KRUN + 4 * ks + e;
+    }
+}
+
+// B fragment (K^T) of k-step ks from the lane's K code run.
+template <int DT, int NW>
+__device__ __forceinline__ void kfrag(const uint32_t (&kw)[NW], int ks, uint32_t& b0, uint32_t& b1)
+{
+    if constexpr (DT == PKV_INT8) {
+        const uint32_t w = kw[ks] ^ 0x80808080u;
+        b0 = i8x2(w, 0x4140);
+        b1 = i8x2(w, 0x4342);
+    } else if constexpr (DT == PKV_FP8E4M3) {
+        b0 = e4m3x2(kw[ks]);
+        b1 = e4m3x2(kw[ks] >> 16);
+    } else {
+        const uint32_t w = kw[ks >> 1] ^ 0x88888888u;
+        b0 = i4x2(w, (ks & 1) * 2);
+        b1 = i4x2(w, (ks & 1) * 2 + 1);
+    }
+}
+
+// A fragments (V^T) for the m-tiles one word of the lane's V run covers.  ab / cd are
+// the words of token rows (2qd, 2qd+1) and (2qd+8, 2qd+9); va[j] gets m-tile j of the word.
+template <int DT>
+__device__ __forceinline__ void vfrags(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t (&va)[4][4])
+{
+    if constexpr (DT == PKV_INT4) {
+        const uint32_t ab0 = __byte_perm(a, b, 0x5410) ^ 0x88888888u, ab1 = __byte_perm(a, b, 0x7632) ^ 0x88888888u;
+        const uint32_t cd0 = __byte_perm(c, d, 0x5410) ^ 0x88888888u, cd1 = __byte_perm(c, d, 0x7632) ^ 0x88888888u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t ab = j < 2 ? ab0 : ab1, cd = j < 2 ? cd0 : cd1;
+            const int s = (j & 1) * 2;
+            va[j][0] = i4x2(ab, s);
+            va[j][1] = i4x2(ab, s + 1);
+            va[j][2] = i4x2(cd, s);
+            va[j][3] = i4x2(cd, s + 1);
+        }
+    } else {
+        const uint32_t ab_lo = __byte_perm(a, b, 0x5140), ab_hi = __byte_perm(a, b, 0x7362);
+        const uint32_t cd_lo = __byte_perm(c, d, 0x5140), cd_hi = __byte_perm(c, d, 0x7362);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint32_t ab = j ? ab_hi : ab_lo, cd = j ? cd_hi : cd_lo;
+            if constexpr (DT == PKV_INT8) {
+                va[j][0] = i8x2(ab ^ 0x80808080u, 0x4140);
+                va[j][1] = i8x2(ab ^ 0x80808080u, 0x4342);
+                va[j][2] = i8x2(cd ^ 0x80808080u, 0x4140);
+                va[j][3] = i8x2(cd ^ 0x80808080u, 0x4342);
+            } else {
+                va[j][0] = e4m3x2(ab);
+                va[j][1] = e4m3x2(ab >> 16);
+                va[j][2] = e4m3x2(cd);
+                va[j][3] = e4m3x2(cd >> 16);
+            }
+        }
+    }
+}
+
+template <int DT, int D, int NHT>
+__global__ void __launch_bounds__(32)
+decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV)
+{
+    using Cfg = QCfg<DT, D>;
+    constexpr int STAGES = Cfg::STAGES;
+    constexpr int ROW = Cfg::ROW, SWZ = Cfg::SWZ;
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ __align__(8) uint64_t bars[STAGES];
+    __shared__ int tbl[kMaxPartTiles];
+    __shared__ float2 tsc[kMaxPartTiles];   // (K scale, V scale) of each tile
+
+    const int lane = threadIdx.x;
+    const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int r = lane >> 2, qd = lane & 3;
+    const int hbase = g * p.G;
+
+    const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
+    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
+    const int tok0 = part * p.part_tokens;
+    if (tok0 >= ctx) {
+        if (part == 0) {
+            float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
+            for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
+        }
+        return;
+    }
+    const int ntok = min(p.part_tokens, ctx - tok0);
+    const int ntiles = (ntok + kBlock - 1) / kBlock;
+
+    const int32_t* trow = p.tables + (size_t)b * p.W + tok0 / kBlock;
+    for (int j = lane; j < ntiles; j += 32) {
+        int blk = trow[j];
+        if ((unsigned)blk >= (unsigned)p.N) {
+            flag_status(p.status, PKV_DEV_BAD_BLOCK);
+            blk = 0;
+        }
+        tbl[j] = blk;
+        const size_t si = (size_t)blk * p.H_kv + g;
+        tsc[j] = make_float2(p.k_scale[si], p.v_scale[si]);
+    }
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    if (lane == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        mbar_fence_init();
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    __syncwarp();
+
+    auto issue = [&](int j) {
+        const int s = j % STAGES;
+        const uint32_t bar = smem_u32(&bars[s]);
+        const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
+        const int row = (tbl[j] * p.H_kv + g) * kBlock;
+        mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        tma_load_2d(kdst, &tmK, 0, row, bar);
+        tma_load_2d(kdst + Cfg::TILE, &tmV, 0, row, bar);
+    };
+    if (lane == 0) {
+        for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
+    }
+
+    // q as fp16 A fragments, k-slots assigned to physical dims by kdim()
+    uint32_t qa[Cfg::KS][4];
+    {
+        const bool bf = p.q_bf16;
+        const uint16_t* qh = static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D;
+        auto qv = [&](int row, int dim) -> float {
+            const uint16_t u = __ldg(qh + row * D + dim);
+            return bf ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
+        };
+        const bool r0 = r < p.G, r1 = (NHT == 2) && (r + 8 < p.G);
+#pragma unroll
+        for (int ks = 0; ks < Cfg::KS; ++ks) {
+            const int d0 = kdim<DT, D>(ks, qd, 0), d1 = kdim<DT, D>(ks, qd, 1);
+            const int d2 = kdim<DT, D>(ks, qd, 2), d3 = kdim<DT, D>(ks, qd, 3);
+            qa[ks][0] = r0 ? pack2<false>(qv(r, d0), qv(r, d1)) : 0u;
+            qa[ks][2] = r0 ? pack2<false>(qv(r, d2), qv(r, d3)) : 0u;
+            qa[ks][1] = r1 ? pack2<false>(qv(r + 8, d0), qv(r + 8, d1)) : 0u;
+            qa[ks][3] = r1 ? pack2<false>(qv(r + 8, d2), qv(r + 8, d3)) : 0u;
+        }
+    }
+
+    float o[Cfg::MT][NHT][4];
+#pragma unroll
+    for (int mt = 0; mt < Cfg::MT; ++mt)
+#pragma unroll
+        for (int hn = 0; hn < NHT; ++hn)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[mt][hn][c] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+
+    int j = 0;
+    bool ok = true;
+    for (; j < ntiles; ++j) {
+        const int s = j % STAGES;
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1)) {
+            ok = false;
+            break;
+        }
+        const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
+        const uint32_t vb = kb + Cfg::TILE;
+        const int nv = min(kBlock, ntok - j * kBlock);
+        const float2 sc_kv = tsc[j];
+
+        // S = Q . K^T, token 8 nt + r of the tile in n-tile nt
+        float sc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
+            uint32_t kw[Cfg::KRUN / 4];
+            load_run<ROW, SWZ, Cfg::KRUN>(kw, kb, nt * 8 + r, qd * Cfg::KRUN);
+#pragma unroll
+            for (int ks = 0; ks < Cfg::KS; ++ks) {
+                uint32_t b0, b1;
+                kfrag<DT>(kw, ks, b0, b1);
+                mma16816<false>(sc[nt], qa[ks], b0, b1);
+            }
+        }
+
+        const float sl = p.scale_log2 * sc_kv.x;
+        float pr[2][4];
+        float alpha[2];
+#pragma unroll
+        for (int hr = 0; hr < NHT; ++hr) {
+            float x[2][2];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tok = nt * 8 + 2 * qd + e;
+                    x[nt][e] = tok < nv ? sc[nt][2 * hr + e] * sl : -INFINITY;
+                    mx = fmaxf(mx, x[nt][e]);
+                }
+            mx = warp_max_quad(mx);
+            const float mn = fmaxf(m_run[hr], mx);
+            alpha[hr] = ex2(m_run[hr] - mn);
+            float sum = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    pr[nt][2 * hr + e] = ex2(x[nt][e] - mn);
+                    sum += pr[nt][2 * hr + e];
+                }
+            l_run[hr] = l_run[hr] * alpha[hr] + sum;
+            m_run[hr] = mn;
+        }
+        const bool moved = (alpha[0] != 1.f) || (NHT == 2 && alpha[1] != 1.f);
+        if (__any_sync(0xffffffffu, moved)) {
+#pragma unroll
+            for (int hn = 0; hn < NHT; ++hn) {
+                const float a_lo = __shfl_sync(0xffffffffu, alpha[hn], 8 * qd);
+                const float a_hi = __shfl_sync(0xffffffffu, alpha[hn], 8 * qd + 4);
+#pragma unroll
+                for (int mt = 0; mt < Cfg::MT; ++mt) {
+                    o[mt][hn][0] *= a_lo;
+                    o[mt][hn][1] *= a_hi;
+                    o[mt][hn][2] *= a_lo;
+                    o[mt][hn][3] *= a_hi;
+                }
+            }
+        }
+
+        // P^T (times the tile's V scale) as fp16 hi + lo B fragments
+        uint32_t bh[NHT][2], bl[NHT][2];
+#pragma unroll
+        for (int hn = 0; hn < NHT; ++hn)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float p0 = pr[nt][2 * hn] * sc_kv.y, p1 = pr[nt][2 * hn + 1] * sc_kv.y;
+                bh[hn][nt] = pack2<false>(p0, p1);
+                const float2 back = unpack2<false>(bh[hn][nt]);
+                bl[hn][nt] = pack2<false>(p0 - back.x, p1 - back.y);
+            }
+
+        uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
+        if (nv < kBlock) {
+            keep01 = (2 * qd < nv ? 0x0000ffffu : 0u) | (2 * qd + 1 < nv ? 0xffff0000u : 0u);
+            keep23 = (8 + 2 * qd < nv ? 0x0000ffffu : 0u) | (9 + 2 * qd < nv ? 0xffff0000u : 0u);
+        }
+        uint32_t wa[Cfg::VRUN / 4], wb[Cfg::VRUN / 4], wc[Cfg::VRUN / 4], wd[Cfg::VRUN / 4];
+        load_run<ROW, SWZ, Cfg::VRUN>(wa, vb, 2 * qd, r * Cfg::VRUN);
+        load_run<ROW, SWZ, Cfg::VRUN>(wb, vb, 2 * qd + 1, r * Cfg::VRUN);
+        load_run<ROW, SWZ, Cfg::VRUN>(wc, vb, 2 * qd + 8, r * Cfg::VRUN);
+        load_run<ROW, SWZ, Cfg::VRUN>(wd, vb, 2 * qd + 9, r * Cfg::VRUN);
+        constexpr int MT_PER_WORD = DT == PKV_INT4 ? 4 : 2;
+#pragma unroll
+        for (int k = 0; k < Cfg::VRUN / 4; ++k) {
+            uint32_t va[4][4];
+            vfrags<DT>(wa[k], wb[k], wc[k], wd[k], va);
+#pragma unroll
+            for (int jj = 0; jj < MT_PER_WORD; ++jj) {
+                const int mt = k * MT_PER_WORD + jj;
+                va[jj][0] &= keep01;
+                va[jj][1] &= keep01;
+                va[jj][2] &= keep23;
+                va[jj][3] &= keep23;
+#pragma unroll
+                for (int hn = 0; hn < NHT; ++hn) {
+                    mma16816<false>(o[mt][hn], va[jj], bh[hn][0], bh[hn][1]);
+                    mma16816<false>(o[mt][hn], va[jj], bl[hn][0], bl[hn][1]);
+                }
+            }
+        }
+
+        __syncwarp();
+        if (lane == 0 && j + STAGES < ntiles) {
+            fence_proxy_async_smem();
+            issue(j + STAGES);
+        }
+    }
+
+    if (!ok) {
+        if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
+        for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
+            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
+        return;
+    }
+
+    // ---- epilogue: O^T row (D/8) r + 2 mt (+1 for the second half) -> [head][dim]
+#pragma unroll
+    for (int hr = 0; hr < NHT; ++hr) l_run[hr] = warp_sum_quad(l_run[hr]);
+    const bool final_out = (nparts == 1);
+    float* so = reinterpret_cast<float*>(smem);
+    constexpr int SR = D + 4;
+    __syncwarp();
+#pragma unroll
+    for (int hn = 0; hn < NHT; ++hn) {
+        float inv_lo = 1.f, inv_hi = 1.f;
+        const float la = __shfl_sync(0xffffffffu, l_run[hn], 8 * qd);
+        const float lb = __shfl_sync(0xffffffffu, l_run[hn], 8 * qd + 4);
+        if (final_out) {
+            inv_lo = 1.f / la;
+            inv_hi = 1.f / lb;
+        }
+        const int h0 = 8 * hn + 2 * qd;
+#pragma unroll
+        for (int mt = 0; mt < Cfg::MT; ++mt) {
+            const int d0 = (D / 8) * r + 2 * mt;
+            so[h0 * SR + d0] = o[mt][hn][0] * inv_lo;
+            so[(h0 + 1) * SR + d0] = o[mt][hn][1] * inv_hi;
+            so[h0 * SR + d0 + 1] = o[mt][hn][2] * inv_lo;
+            so[(h0 + 1) * SR + d0 + 1] = o[mt][hn][3] * inv_hi;
+        }
+    }
+    __syncwarp();
+    const size_t row0 = (size_t)b * p.H_q + hbase;
+    float* dst = final_out ? p.out : p.ws_o;
+    for (int i = lane; i < p.G * (D / 4); i += 32) {
+        const int h = i / (D / 4), c4 = i % (D / 4);
+        const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
+        const size_t off = final_out ? (row0 + h) * D : ((row0 + h) * p.max_parts + part) * D;
+        *reinterpret_cast<float4*>(dst + off + 4 * c4) = v;
+    }
+    if (!final_out && qd == 0) {
+#pragma unroll
+        for (int hr = 0; hr < NHT; ++hr) {
+            const int h = r + 8 * hr;
+            if (h < p.G)
+                *reinterpret_cast<float2*>(p.ws_ml + ((row0 + h) * p.max_parts + part) * 2) =
+                    make_float2(m_run[hr], l_run[hr]);
+        }
+    }
+}
+
+template <int DT, int D>
+int launch_q(const DecodeParams& p, int nht, dim3 grid, cudaStream_t s, const CUtensorMap* tmk, const CUtensorMap* tmv)
+{
+    constexpr int smem = QCfg<DT, D>::SMEM;
+    auto k1 = decode_mmaq_kernel<DT, D, 1>;
+    auto k2 = decode_mmaq_kernel<DT, D, 2>;
+    auto kern = nht == 1 ? k1 : k2;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    kern<<<grid, 32, smem, s>>>(p, *tmk, *tmv);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,
+                        const CUtensorMap* tmk, const CUtensorMap* tmv)
+{
+    switch (kv_dtype * 1000 + d) {
+    case PKV_INT8 * 1000 + 128: return launch_q<PKV_INT8, 128>(p, nht, grid, s, tmk, tmv);
+    case PKV_INT8 * 1000 + 64: return launch_q<PKV_INT8, 64>(p, nht, grid, s, tmk, tmv);
+    case PKV_FP8E4M3 * 1000 + 128: return launch_q<PKV_FP8E4M3, 128>(p, nht, grid, s, tmk, tmv);
+    case PKV_FP8E4M3 * 1000 + 64: return launch_q<PKV_FP8E4M3, 64>(p, nht, grid, s, tmk, tmv);
+    case PKV_INT4 * 1000 + 128: return launch_q<PKV_INT4, 128>(p, nht, grid, s, tmk, tmv);
+    case PKV_INT4 * 1000 + 64: return launch_q<PKV_INT4, 64>(p, nht, grid, s, tmk, tmv);
+    default: return PKV_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace pkv
