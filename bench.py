@@ -1,18 +1,26 @@
-"""Benchmark: paged GQA decode over a paged KV cache on B200.
+"""Benchmark: attention over a paged KV cache on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gqa70b|llama8b|prefix_chunk|quant_int8|...]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the CPU oracle on this host's cores
 
-A step is one pass of the hot path over one batch: for every layer, kv_append of each
-sequence's new token followed by paged_decode_attn over the whole cached context.
-Default workload: the 70B-class GQA decode -- 80 layers, 64 query heads, 8 KV heads,
-head dim 128, bf16 K/V, 170 sequences with contexts ~ N(3000, 400) clipped to
-[1024, 4096], block tables permuted over a pool of 170 x 256 blocks per layer.
+A step is one pass of the hot path over one batch.  Default workload (`gqa70b`): the
+70B-class GQA decode -- 80 layers, 64 query heads, 8 KV heads, head dim 128, bf16 K/V,
+170 sequences with contexts ~ N(3000, 400) clipped to [1024, 4096], block tables
+permuted over a pool of 170 x 256 blocks per layer; per layer, kv_append of every
+sequence's new token, then paged_decode_attn over its whole cached context.
 
-Prints ONE JSON line (rank 0).  `value` is KV GB/s (algorithmic K/V bytes read by the
-decode calls of all ranks / the max-over-ranks device time of the K timed steps).
-With --gpus N > 1 (torchrun), every rank runs an independent replica: the path has no
-data exchange, so there is no collective beyond the timing barrier.
+Other workloads (one JSON line each): `llama8b` (1 layer, B 64, H_q 32, ctx U[512, 4096]);
+`quant_int8` / `quant_fp8` / `quant_int4` / `quant_bf16` (1 layer, B 16, H_q 64, H_kv 8,
+ctx U[32768, 131072], K/V stored quantized with one fp32 scale per (block, head), bf16
+N(0,1) source with 1% outlier channels x8; `quant_bf16` is the unquantized control);
+`prefix_chunk` (1 layer of the 70B shape: 256 decodes sharing a 4,000-token prefix plus
+private 200-token suffixes and 0-300 decoded tokens, and one 512-token prefill chunk of
+a new request over the same prefix, in every step).
+
+Prints ONE JSON line (rank 0).  `value` is KV GB/s: the K/V bytes the step's attention
+calls read (logically, per sequence) / the max-over-ranks device time of the K timed
+steps.  With --gpus N > 1 (torchrun), every rank runs an independent replica (the path
+has no data exchange), so there is no collective beyond the timing barrier.
 """
 from __future__ import annotations
 
@@ -20,7 +28,6 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -37,6 +44,9 @@ from paged_kv_cache_431_b200 import workloads as wl  # noqa: E402
 
 METRIC = "paged GQA decode: KV HBM GB/s (% of ~8 TB/s peak); seq-tokens/s per layer"
 PROFILES = os.path.join(ROOT, "profiles")
+DECODE_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_quant.cu",
+               "paged_kv_cache_431_b200/csrc/decode_common.cuh", "paged_kv_cache_431_b200/csrc/common.cuh"]
+PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
 
 
 # ------------------------------------------------------------------ utils --
@@ -49,9 +59,9 @@ def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return p, "measured"
     except Exception:
-        return 6650.0, "fallback"
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
 class ClockSampler:
@@ -70,7 +80,7 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -103,26 +113,6 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_traffic(kernel_key: str, src_files):
-    """DRAM bytes per launch from a committed ncu summary, only if the kernel sources are
-    unchanged since the capture (their hash is stored with the figure)."""
-    path = os.path.join(PROFILES, "traffic.json")
-    try:
-        with open(path) as f:
-            rec = json.load(f).get(kernel_key)
-    except Exception:
-        return None
-    if not rec:
-        return None
-    h = hashlib.sha256()
-    for s in src_files:
-        with open(os.path.join(ROOT, s), "rb") as f:
-            h.update(f.read())
-    if rec.get("src_sha256") != h.hexdigest():
-        return None
-    return rec.get("bytes_per_launch")
-
-
 def source_hash(src_files):
     h = hashlib.sha256()
     for s in src_files:
@@ -131,184 +121,147 @@ def source_hash(src_files):
     return h.hexdigest()
 
 
-DECODE_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
+def kernel_traffic(key: str, src_files):
+    """DRAM bytes per launch from a committed ncu summary, used only while the kernel
+    sources still hash to the version that was captured."""
+    try:
+        with open(os.path.join(PROFILES, "traffic.json")) as f:
+            rec = json.load(f).get(key)
+    except Exception:
+        return None
+    if not rec or rec.get("src_sha256") != source_hash(src_files):
+        return None
+    return rec.get("bytes_per_launch")
 
 
 # -------------------------------------------------------------- workloads --
 
+QUANT_DESC = ("quantized long-context decode, 1 layer: H_q 64, H_kv 8, d 128, B 16, ctx ~ U[32768, 131072], "
+              "bf16 N(0,1) source with 1% outlier channels x8, stored as {}, one fp32 scale per (block, kv head)")
 WORKLOADS = {
-    "gqa70b": dict(layers=80, B=170, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=256,
+    "gqa70b": dict(kind="decode", layers=80, B=170, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=256,
+                   lens="gqa70b", pool_blocks=170 * 256,
                    desc="70B-class GQA decode: 80 layers, H_q 64, H_kv 8, d 128, bf16, B 170, "
                         "ctx ~ N(3000, 400) clipped to [1024, 4096], pool 170 x 256 blocks per layer"),
-    "llama8b": dict(layers=1, B=64, H_q=32, H_kv=8, d=128, dtype=wl.BF16, width=256,
+    "llama8b": dict(kind="decode", layers=1, B=64, H_q=32, H_kv=8, d=128, dtype=wl.BF16, width=256,
+                    lens="llama8b", pool_blocks=64 * 256,
                     desc="Llama-3-8B-shaped decode, 1 layer: H_q 32, H_kv 8, d 128, bf16, B 64, "
                          "ctx ~ U[512, 4096], pool for 64 x 4096 tokens"),
+    "quant_int8": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.INT8, width=8192,
+                       lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("int8")),
+    "quant_fp8": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.FP8, width=8192,
+                      lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("fp8 e4m3")),
+    "quant_int4": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.INT4, width=8192,
+                       lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("packed int4")),
+    "quant_bf16": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=8192,
+                       lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("bf16 (control)")),
+    "prefix_chunk": dict(kind="prefix", layers=1, B=256, H_q=64, H_kv=8, d=128, dtype=wl.BF16,
+                         desc="prefix sharing + chunked prefill, 1 layer of the 70B shape, bf16: 256 decodes "
+                              "share a 4,000-token prefix (250 blocks) + private 200-token suffixes + U{0..300} "
+                              "decoded tokens; plus one 512-token causal prefill chunk of a new request over "
+                              "the prefix"),
 }
+ELEM_BYTES = {wl.F16: 2.0, wl.BF16: 2.0, wl.INT8: 1.0, wl.FP8: 1.0, wl.INT4: 0.5}
+DTYPE_NAME = {wl.F16: "f16", wl.BF16: "bf16", wl.INT8: "int8", wl.FP8: "fp8e4m3", wl.INT4: "int4"}
 
 
-def make_lens(name, gen, B):
-    if name == "gqa70b":
-        return wl.gqa70b_lens(gen, B)
-    if name == "llama8b":
-        return wl.llama8b_lens(gen, B)
-    raise ValueError(name)
+def make_lens(kind, gen, B):
+    return {"gqa70b": wl.gqa70b_lens, "llama8b": wl.llama8b_lens, "quant": wl.quant_long_lens}[kind](gen, B)
 
 
-def algorithmic_bytes(ctx_lens, B, H_q, H_kv, d, elem_bytes):
-    """Bytes a decode call must move: every cached K and V element once, plus q, out,
-    the used block-table entries and the context lengths."""
+def decode_bytes(ctx_lens, B, H_q, H_kv, d, dt):
+    """(K/V bytes, all algorithmic bytes) of one decode call: every cached K and V
+    element once (and its block's scales), plus q, out, used table entries, lengths."""
     sum_ctx = int(ctx_lens.sum())
-    kv = sum_ctx * 2 * H_kv * d * elem_bytes
     blocks = int(sum(wl.ceil_div(int(n), 16) for n in ctx_lens))
-    other = B * H_q * d * elem_bytes + B * H_q * d * 4 + blocks * 4 + B * 4
-    return kv, kv + other
+    kv = int(sum_ctx * 2 * H_kv * d * ELEM_BYTES[dt])
+    scales = blocks * H_kv * 2 * 4 if dt in (wl.INT8, wl.FP8, wl.INT4) else 0
+    other = B * H_q * d * 2 + B * H_q * d * 4 + blocks * 4 + B * 4
+    return kv, kv + scales + other
 
 
 # ------------------------------------------------------------- GPU arm --
 
-def run_gpu(args):
+class Timed:
+    """Device timing of the K steps plus per-call events around the dominant calls."""
+
+    def __init__(self, steps, per_step):
+        mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        self.ev = [[(mk(), mk()) for _ in range(per_step)] for _ in range(steps)]
+
+    def call_ms(self):
+        return [a.elapsed_time(b) for st in self.ev for (a, b) in st]
+
+
+def build_decode(args, cfg, dev, rank):
     from paged_kv_cache_431_b200 import pkv
 
-    rank, local_rank, world = dist_env()
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    dev = torch.device("cuda", local_rank if world > 1 else 0)
-    torch.cuda.set_device(dev)
-    cfg = WORKLOADS[args.workload]
     L, B, H_q, H_kv, d, dt = cfg["layers"], cfg["B"], cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
-    tdt = wl.TORCH_DTYPE[dt]
-    elem = 2
-
     gen = wl.generator(431 + 3 + rank)
-    ctx = make_lens(args.workload, gen, B)
-    N = B * cfg["width"]
+    ctx = make_lens(cfg["lens"], gen, B)
+    N = cfg["pool_blocks"]
     paging = wl.allocate(ctx, N, cfg["width"], gen)
-    per_layer_pool = 2 * N * H_kv * 16 * d * elem
+    quant = dt in (wl.INT8, wl.FP8, wl.INT4)
+    per_layer_pool = 2 * N * H_kv * 16 * d * ELEM_BYTES[dt]
     free, _ = torch.cuda.mem_get_info(dev)
     L_phys = max(1, min(L, int(args.pool_fraction * free // per_layer_pool)))
     gd = wl.generator(431 + 100 + rank, dev)
-    k_pool = torch.empty(L_phys, N, H_kv, 16, d, dtype=tdt, device=dev)
-    v_pool = torch.empty_like(k_pool)
-    for l in range(L_phys):
-        k_pool[l] = wl.normal((N, H_kv, 16, d), tdt, gd, dev)
-        v_pool[l] = wl.normal((N, H_kv, 16, d), tdt, gd, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    pool = pkv.KVPool(k_pool, v_pool, dt, d, device_status=status)
+    if not quant:
+        tdt = wl.TORCH_DTYPE[dt]
+        k_pool = torch.empty(L_phys, N, H_kv, 16, d, dtype=tdt, device=dev)
+        v_pool = torch.empty_like(k_pool)
+        for l in range(L_phys):
+            k_pool[l] = wl.normal((N, H_kv, 16, d), tdt, gd, dev)
+            v_pool[l] = wl.normal((N, H_kv, 16, d), tdt, gd, dev)
+        pool = pkv.KVPool(k_pool, v_pool, dt, d, device_status=status)
+        src_dtype = tdt
+    else:
+        pool = pkv.KVPool.allocate(L_phys, N, H_kv, d, dt)
+        out_ch = wl.outlier_channels(gen, H_kv, d)
+        for l in range(L_phys):           # bulk fill through kv_append (untimed)
+            for b in range(B):
+                n = int(ctx[b])
+                k, v = wl.kv_source(n, H_kv, d, gd, dev, outliers=out_ch)
+                pkv.kv_append(pool, l, k, v, wl.slots_for(paging.tables, [b] * n, torch.arange(n)).to(dev))
+                del k, v
+        src_dtype = torch.bfloat16
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
 
     tables = paging.tables.to(dev)
     ctx_d = ctx.to(dev)
     max_ctx = int(ctx.max())
     slots = wl.slots_for(paging.tables, range(B), (ctx - 1).long()).to(dev)   # each step's new token
-    q = wl.normal((L, B, H_q, d), tdt, gd, dev)
-    k_new = wl.normal((L, B, H_kv, d), tdt, gd, dev)
-    v_new = wl.normal((L, B, H_kv, d), tdt, gd, dev)
+    q = wl.normal((L, B, H_q, d), src_dtype, gd, dev)
+    k_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
+    v_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     out = torch.empty(L, B, H_q, d, dtype=torch.float32, device=dev)
-    ws_bytes = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx), 16), dtype=torch.uint8,
+                     device=dev)
+    aws = torch.empty(max(pkv.kv_append_workspace_bytes(pool, B), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    scale = d ** -0.5
 
     def step(ev=None):
         for l in range(L):
             lp = l % L_phys
-            pkv.kv_append(pool, lp, k_new[l], v_new[l], slots)
+            pkv.kv_append(pool, lp, k_new[l], v_new[l], slots, workspace=aws)
             if ev is not None:
                 ev[l][0].record(stream)
-            pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, d ** -0.5, max_ctx, out=out[l], workspace=ws)
+            pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws)
             if ev is not None:
                 ev[l][1].record(stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if pkv.read_device_status(pool):
-        raise RuntimeError("device status set during warm-up")
+    kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt)
+    parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx) > 0
+    launches = L * ((3 if quant else 1) + 1 + (1 if parts else 0))
 
-    kv_bytes, alg_bytes = algorithmic_bytes(ctx, B, H_q, H_kv, d, elem)
-    call_events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
-                   for _ in range(args.steps)]
-    clocks = ClockSampler(dev.index)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for s in range(args.steps):
-        step(call_events[s])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    clk = clocks.stop()
-    if world > 1:
-        torch.distributed.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    call_ms = [e0.elapsed_time(e1) for st in call_events for (e0, e1) in st]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-    if pkv.read_device_status(pool):
-        raise RuntimeError("device status set during timing")
-
-    ms_per_step = elapsed_ms / args.steps
-    total_kv = kv_bytes * L * args.steps * world
-    value = total_kv / (elapsed_ms * 1e-3) / 1e9
-    seq_tokens_per_s_layer = int(ctx.sum()) * L * args.steps * world / (elapsed_ms * 1e-3) / L
-    peak, peak_kind = measured_peaks()
-    avg_call_s = statistics.mean(call_ms) * 1e-3
-    achieved = alg_bytes / avg_call_s / 1e9
-    traffic = kernel_traffic(f"decode_mma16_{args.workload}", DECODE_SRCS)
-    launches_per_layer = 2 + (1 if ws_bytes > 0 else 0)
-
-    e2e = run_e2e(args, pool, L, L_phys, B, H_q, H_kv, d, tdt, paging, ctx, max_ctx, kv_bytes, world, dev)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(pool, paging, ctx, H_q, H_kv, d, dt, q[0], budget_s=args.cpu_seconds)
-
-    res = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "description": cfg["desc"], "layers": L, "batch": B,
-                   "q_heads": H_q, "kv_heads": H_kv, "head_dim": d, "sum_ctx": int(ctx.sum()),
-                   "physical_layer_pools": L_phys, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: each decode call reads {kv_bytes / 1e9:.2f} GB of K/V",
-                   "partition_tokens": "auto"},
-        "seq_tokens_per_s_per_layer": round(seq_tokens_per_s_layer),
-        "pct_of_8tbs_nominal": round(100 * value / world / 8000.0, 1),
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_attn (main + split-K merge)",
-                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
-                     "avg_launch_us": round(avg_call_s * 1e6, 2)},
-        "e2e": e2e,
-        "gpu_launches": args.steps * L * launches_per_layer,
-        "clocks": clk,
-    }
-    if cpu is not None:
-        res["cpu_baseline"] = cpu
-    if rank == 0:
-        print(json.dumps(res), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
-
-
-def run_e2e(args, pool, L, L_phys, B, H_q, H_kv, d, tdt, paging, ctx, max_ctx, kv_bytes, world, dev):
-    """The same step through the C-ABI with host buffers: every step copies each layer's
-    q and new K/V (and the block tables, context lengths and slots) from pinned host
-    memory and reads every layer's attention output back.  Copies run on two copy
-    streams overlapped with the kernels of neighbouring layers."""
-    from paged_kv_cache_431_b200 import pkv
-
+    # host-buffer (e2e) step: inputs from pinned memory, every layer's output read back
     g = wl.generator(999)
-    hq = wl.normal((L, B, H_q, d), tdt, g).pin_memory()
-    hk = wl.normal((L, B, H_kv, d), tdt, g).pin_memory()
-    hv = wl.normal((L, B, H_kv, d), tdt, g).pin_memory()
+    hq = wl.normal((L, B, H_q, d), src_dtype, g).pin_memory()
+    hk = wl.normal((L, B, H_kv, d), src_dtype, g).pin_memory()
+    hv = wl.normal((L, B, H_kv, d), src_dtype, g).pin_memory()
     htab = paging.tables.clone().pin_memory()
     hctx = ctx.clone().pin_memory()
     hslots = wl.slots_for(paging.tables, range(B), (ctx - 1).long()).pin_memory()
@@ -316,14 +269,12 @@ def run_e2e(args, pool, L, L_phys, B, H_q, H_kv, d, tdt, paging, ctx, max_ctx, k
     dq, dk, dv = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
     dtab, dctx, dslots = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (htab, hctx, hslots))
     dout = torch.empty(hout.shape, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx), 16), dtype=torch.uint8, device=dev)
-    comp = torch.cuda.current_stream(dev)
     h2d = torch.cuda.Stream(dev)
     d2h = torch.cuda.Stream(dev)
 
-    def step():
+    def e2e_step():
         start = torch.cuda.Event()
-        start.record(comp)
+        start.record(stream)
         h2d.wait_event(start)
         ready = []
         with torch.cuda.stream(h2d):
@@ -339,11 +290,11 @@ def run_e2e(args, pool, L, L_phys, B, H_q, H_kv, d, tdt, paging, ctx, max_ctx, k
                 ready.append(e)
         done = []
         for l in range(L):
-            comp.wait_event(ready[l])
-            pkv.kv_append(pool, l % L_phys, dk[l], dv[l], dslots)
-            pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, d ** -0.5, max_ctx, out=dout[l], workspace=ws)
+            stream.wait_event(ready[l])
+            pkv.kv_append(pool, l % L_phys, dk[l], dv[l], dslots, workspace=aws)
+            pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, scale, max_ctx, out=dout[l], workspace=ws)
             e = torch.cuda.Event()
-            e.record(comp)
+            e.record(stream)
             done.append(e)
         with torch.cuda.stream(d2h):
             for l in range(L):
@@ -351,118 +302,292 @@ def run_e2e(args, pool, L, L_phys, B, H_q, H_kv, d, tdt, paging, ctx, max_ctx, k
                 hout[l].copy_(dout[l], non_blocking=True)
         fin = torch.cuda.Event()
         fin.record(d2h)
-        comp.wait_event(fin)
+        stream.wait_event(fin)
 
-    for _ in range(max(1, args.warmup)):
-        step()
-    torch.cuda.synchronize(dev)
+    h2d_bytes = sum(t.numel() * t.element_size() for t in (hq, hk, hv, htab, hctx, hslots))
+    d2h_bytes = hout.numel() * hout.element_size()
+    peaks, kind = measured_peaks()
+    info = dict(
+        config={"workload": args.workload, "description": cfg["desc"], "layers": L, "batch": B, "q_heads": H_q,
+                "kv_heads": H_kv, "head_dim": d, "kv_dtype": DTYPE_NAME[dt], "sum_ctx": int(ctx.sum()),
+                "physical_layer_pools": L_phys, "parallelism": "replicas",
+                "l2": f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V",
+                "partition_tokens": "auto"},
+        kv_bytes_per_step=kv * L, seq_tokens_per_step=int(ctx.sum()) * L, layers=L,
+        roofline=dict(bound="hbm", kernel="paged_decode_attn (main + split-K merge)", alg_bytes=alg,
+                      peak=float(peaks["hbm_gbs"]), unit="GB/s",
+                      peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
+                      traffic=kernel_traffic(f"decode_{args.workload}", DECODE_SRCS)),
+        launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",
+        h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L)
+    return step, e2e_step, info, pool
+
+
+def build_prefix_chunk(args, cfg, dev, rank):
+    """Config 4: one step = 256 decode appends + decode over prefix-sharing tables, then
+    the new request's 512-token chunk append + chunked prefill over the same prefix."""
+    from paged_kv_cache_431_b200 import pkv
+
+    B, H_q, H_kv, d = cfg["B"], cfg["H_q"], cfg["H_kv"], cfg["d"]
+    P0, C, pre_blocks = 4000, 512, 250
+    gen = wl.generator(431 + 4 + rank)
+    n_dec = torch.randint(0, 301, (B,), generator=gen, dtype=torch.int32)
+    ctx = (P0 + 200 + n_dec + 1).to(torch.int32)           # includes this step's token
+    lens_all = torch.cat([ctx, torch.tensor([P0 + C], dtype=torch.int32)])
+    N = pre_blocks + B * 32 + 32 + 64
+    width = wl.ceil_div(int(lens_all.max()), 16)
+    paging = wl.allocate(lens_all, N, width, gen, shared_prefix_blocks=pre_blocks)
+    gd = wl.generator(431 + 200 + rank, dev)
+    k_pool = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, dev)
+    v_pool = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, dev)
+    pool = pkv.KVPool(k_pool, v_pool, wl.BF16, d, device_status=torch.zeros(1, dtype=torch.int32, device=dev))
+    tables = paging.tables[:B].contiguous().to(dev)
+    ctx_d = ctx.to(dev)
+    max_ctx = int(ctx.max())
+    chunk_table = paging.tables[B].contiguous().to(dev)
+    dec_slots = wl.slots_for(paging.tables, range(B), (ctx - 1).long()).to(dev)
+    chunk_slots = wl.slots_for(paging.tables, [B] * C, torch.arange(P0, P0 + C)).to(dev)
+    q_dec = wl.normal((B, H_q, d), torch.bfloat16, gd, dev)
+    k_dec = wl.normal((B, H_kv, d), torch.bfloat16, gd, dev)
+    v_dec = wl.normal((B, H_kv, d), torch.bfloat16, gd, dev)
+    q_chunk = wl.normal((C, H_q, d), torch.bfloat16, gd, dev)
+    k_chunk = wl.normal((C, H_kv, d), torch.bfloat16, gd, dev)
+    v_chunk = wl.normal((C, H_kv, d), torch.bfloat16, gd, dev)
+    out_dec = torch.empty(B, H_q, d, dtype=torch.float32, device=dev)
+    out_chunk = torch.empty(C, H_q, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx), 16), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+    scale = d ** -0.5
+
+    def step(ev=None):
+        pkv.kv_append(pool, 0, k_dec, v_dec, dec_slots)
+        if ev is not None:
+            ev[0][0].record(stream)
+        pkv.paged_decode_attn(pool, 0, q_dec, tables, ctx_d, scale, max_ctx, out=out_dec, workspace=ws)
+        if ev is not None:
+            ev[0][1].record(stream)
+        pkv.kv_append(pool, 0, k_chunk, v_chunk, chunk_slots)
+        if ev is not None:
+            ev[1][0].record(stream)
+        pkv.paged_prefill_chunk_attn(pool, 0, q_chunk, chunk_table, P0, scale, out=out_chunk)
+        if ev is not None:
+            ev[1][1].record(stream)
+
+    dec_kv, dec_alg = decode_bytes(ctx, B, H_q, H_kv, d, wl.BF16)
+    pairs = sum(P0 + i + 1 for i in range(C))                      # causal (query, key) pairs per head
+    flops = 4 * d * pairs * H_q
+    chunk_kv = (P0 + C) * 2 * H_kv * d * 2
+    unique_blocks = int(torch.unique(paging.tables[paging.tables >= 0]).numel())
+
+    hq = torch.cat([q_dec, q_chunk]).cpu().pin_memory()
+    hk = torch.cat([k_dec, k_chunk]).cpu().pin_memory()
+    hv = torch.cat([v_dec, v_chunk]).cpu().pin_memory()
+    hout = torch.empty(B + C, H_q, d, dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (hq, hk, hv))
+    dout = torch.empty(hout.shape, dtype=torch.float32, device=dev)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        pkv.kv_append(pool, 0, dk[:B], dv[:B], dec_slots)
+        pkv.paged_decode_attn(pool, 0, dq[:B], tables, ctx_d, scale, max_ctx, out=dout[:B], workspace=ws)
+        pkv.kv_append(pool, 0, dk[B:], dv[B:], chunk_slots)
+        pkv.paged_prefill_chunk_attn(pool, 0, dq[B:], chunk_table, P0, scale, out=dout[B:])
+        hout.copy_(dout, non_blocking=True)
+
+    peaks, kind = measured_peaks()
+    info = dict(
+        config={"workload": args.workload, "description": cfg["desc"], "decode_batch": B, "q_heads": H_q,
+                "kv_heads": H_kv, "head_dim": d, "prefix_tokens": P0, "chunk_tokens": C,
+                "sum_ctx_decode": int(ctx.sum()), "unique_kv_blocks": unique_blocks,
+                "unique_kv_bytes": unique_blocks * H_kv * 16 * d * 2 * 2,
+                "chunk_gflop": round(flops / 1e9, 2), "parallelism": "replicas",
+                "l2": "steady state, no flush: the shared prefix stays in L2 across the 256 decodes (as in real "
+                      "prefix reuse)"},
+        kv_bytes_per_step=dec_kv + chunk_kv, seq_tokens_per_step=int(ctx.sum()), layers=1,
+        roofline=dict(bound="tensor", kernel="paged_prefill_chunk_attn", alg_flops=flops,
+                      peak=float(peaks["bf16_tflops"]), unit="TFLOP/s",
+                      peak_source=f"{kind} (MEASURED_PEAKS.json bf16_tflops, burst: a short kernel)",
+                      traffic=kernel_traffic("prefill_prefix_chunk", PREFILL_SRCS), call_index=1,
+                      decode_alg_bytes=dec_alg),
+        launches_per_step=4 + (1 if ws.numel() > 16 else 0), dtype="bf16",
+        h2d=sum(t.numel() * t.element_size() for t in (hq, hk, hv)), d2h=hout.numel() * 4, calls_per_step=2)
+    return step, e2e_step, info, pool
+
+
+def time_steps(step, n_steps, per_step_calls, dev, world):
+    timed = Timed(n_steps, per_step_calls)
+    stream = torch.cuda.current_stream(dev)
     if world > 1:
         torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(comp)
-    for _ in range(args.steps):
-        step()
-    t1.record(comp)
+    t0.record(stream)
+    for s in range(n_steps):
+        step(timed.ev[s] if timed is not None else None)
+    t1.record(stream)
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1)
     if world > 1:
         t = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
-    h2d_bytes = sum(t.numel() * t.element_size() for t in (hq, hk, hv, htab, hctx, hslots))
-    d2h_bytes = hout.numel() * hout.element_size()
-    value = kv_bytes * L * args.steps * world / (ms * 1e-3) / 1e9
-    return {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(ms / args.steps, 4),
-            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes}
+    return ms, timed
+
+
+def run_gpu(args):
+    from paged_kv_cache_431_b200 import pkv
+
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    cfg = WORKLOADS[args.workload]
+    builder = build_prefix_chunk if cfg["kind"] == "prefix" else build_decode
+    step, e2e_step, info, pool = builder(args, cfg, dev, rank)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if pkv.read_device_status(pool):
+        raise RuntimeError("device status set during warm-up")
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    elapsed_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world)
+    clk = clocks.stop()
+    if pkv.read_device_status(pool):
+        raise RuntimeError("device status set during timing")
+
+    # end to end through the same calls with host buffers
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms, _ = time_steps(lambda ev=None: e2e_step(), args.steps, 1, dev, world)
+
+    ms_per_step = elapsed_ms / args.steps
+    value = info["kv_bytes_per_step"] * args.steps * world / (elapsed_ms * 1e-3) / 1e9
+    e2e_value = info["kv_bytes_per_step"] * args.steps * world / (e2e_ms * 1e-3) / 1e9
+    call_ms = timed.call_ms()
+    rf = info["roofline"]
+    if rf["bound"] == "hbm":
+        avg_s = statistics.mean(call_ms) * 1e-3
+        achieved = rf["alg_bytes"] / avg_s / 1e9
+        roofline = {"bound": "hbm", "kernel": rf["kernel"], "achieved": round(achieved, 1), "peak": rf["peak"],
+                    "unit": "GB/s", "frac": round(achieved / rf["peak"], 4), "peak_source": rf["peak_source"],
+                    "traffic": rf["traffic"], "algorithmic_bytes_per_launch": rf["alg_bytes"],
+                    "avg_launch_us": round(avg_s * 1e6, 2)}
+    else:
+        ci = rf["call_index"]
+        per_call = [call_ms[i] for i in range(ci, len(call_ms), info["calls_per_step"])]
+        dec_calls = [call_ms[i] for i in range(0, len(call_ms), info["calls_per_step"])]
+        avg_s = statistics.mean(per_call) * 1e-3
+        achieved = rf["alg_flops"] / avg_s / 1e12
+        dec_s = statistics.mean(dec_calls) * 1e-3
+        roofline = {"bound": "tensor", "kernel": rf["kernel"], "achieved": round(achieved, 1), "peak": rf["peak"],
+                    "unit": "TFLOP/s", "frac": round(achieved / rf["peak"], 4), "peak_source": rf["peak_source"],
+                    "traffic": rf["traffic"], "algorithmic_flops_per_launch": rf["alg_flops"],
+                    "avg_launch_us": round(avg_s * 1e6, 2),
+                    "decode_call_us": round(dec_s * 1e6, 2),
+                    "decode_logical_gbs": round(rf["decode_alg_bytes"] / dec_s / 1e9, 1)}
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic",
+        "config": info["config"],
+        "seq_tokens_per_s_per_layer": round(info["seq_tokens_per_step"] / info["layers"] * args.steps * world
+                                            / (elapsed_ms * 1e-3)),
+        "pct_of_8tbs_nominal": round(100 * value / world / 8000.0, 1),
+        "roofline": roofline,
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms / args.steps, 4),
+                "h2d_bytes_per_step": info["h2d"], "d2h_bytes_per_step": info["d2h"]},
+        "gpu_launches": args.steps * info["launches_per_step"],
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_oracle(args.workload, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
 
 
 # ------------------------------------------------------ CPU oracle timing --
 
-def oracle_decode_sample(k_host, v_host, dt, tables, ctx, q_host, seq_ids, H_q, d):
-    """Run the oracle over the given sequences of one layer; returns (seconds, kv bytes)."""
+def cpu_oracle(workload, budget_s=12.0, per_step=None, steps=None, warmup=0):
+    """The oracle as it stands (single-threaded C, fp64) on whole sequences of one layer of
+    the same workload, generated on the host with the same recipe.  With `per_step` it
+    runs warmup + steps steps of `per_step` sequences; otherwise sequences in order until
+    about `budget_s` seconds.  Returns (result dict, list of per-step seconds)."""
     import oracle
-    blocks, sub_t, sub_c = wl.compact_subset(tables, ctx, seq_ids)
-    idx = torch.as_tensor(blocks, dtype=torch.long)
-    kraw = k_host[idx].contiguous().view(torch.int16).numpy().view(np.uint8)
-    vraw = v_host[idx].contiguous().view(torch.int16).numpy().view(np.uint8)
-    opool = oracle.Pool(len(blocks), k_host.shape[1], d, dt, kraw, vraw)
-    qs = q_host[seq_ids]
-    t0 = time.perf_counter()
-    oracle.paged_decode(opool, qs, dt, sub_t, sub_c, np.float32(d ** -0.5))
-    sec = time.perf_counter() - t0
-    kv = int(sub_c.sum()) * 2 * k_host.shape[1] * d * 2
-    return sec, kv
 
-
-def cpu_baseline(pool, paging, ctx, H_q, H_kv, d, dt, q_layer, budget_s=15.0):
-    """The oracle as it stands (single-threaded C, fp64) on a bounded sample of one layer:
-    whole sequences in order until about `budget_s` seconds of CPU work."""
-    k_host = pool.k_data[0].cpu()
-    v_host = pool.v_data[0].cpu()
-    qh = q_layer.cpu()
-    total_s, total_kv, total_tok, seqs = 0.0, 0, 0, 0
-    for b in range(len(ctx)):
-        sec, kv = oracle_decode_sample(k_host, v_host, dt, paging.tables, ctx, qh, [b], H_q, d)
-        total_s += sec
-        total_kv += kv
-        total_tok += int(ctx[b])
-        seqs += 1
-        if total_s >= budget_s:
+    oracle.build()
+    cfg = WORKLOADS[workload]
+    H_q, H_kv, d, dt = cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
+    gen = wl.generator(431 + 3)
+    if cfg["kind"] == "prefix":
+        ctx = (4000 + 200 + torch.randint(0, 301, (cfg["B"],), generator=gen, dtype=torch.int32) + 1)
+    else:
+        ctx = make_lens(cfg["lens"], gen, cfg["B"])
+    gh = wl.generator(431 + 300)
+    quant = dt in (wl.INT8, wl.FP8, wl.INT4)
+    total_s, total_kv, total_tok, seqs, step_secs = 0.0, 0, 0, 0, []
+    n_steps = (warmup + steps) if per_step else 10 ** 9
+    b = 0
+    for s in range(n_steps):
+        ids = [(b + i) % len(ctx) for i in range(per_step or 1)]
+        b += len(ids)
+        step_s = 0.0
+        for sid in ids:
+            n = int(ctx[sid])
+            nb = wl.ceil_div(n, 16)
+            table = torch.arange(nb, dtype=torch.int32).view(1, nb)
+            opool = oracle.Pool(nb, H_kv, d, dt if quant else dt)
+            k, v = wl.kv_source(n, H_kv, d, gh) if quant else (wl.normal((n, H_kv, d), torch.bfloat16, gh),
+                                                              wl.normal((n, H_kv, d), torch.bfloat16, gh))
+            oracle.kv_append(opool, k, v, oracle.BF16, np.arange(n, dtype=np.int32))
+            q = wl.normal((1, H_q, d), torch.bfloat16, gh)
+            t0 = time.perf_counter()
+            oracle.paged_decode(opool, q, oracle.BF16, table, [n], np.float32(d ** -0.5))
+            step_s += time.perf_counter() - t0
+            if s >= warmup:
+                total_kv += int(n * 2 * H_kv * d * ELEM_BYTES[dt])
+                total_tok += n
+                seqs += 1
+        if s >= warmup:
+            total_s += step_s
+            step_secs.append(step_s)
+        if not per_step and total_s >= budget_s:
             break
-    return {"value": round(total_kv / total_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "seq_tokens_per_s_per_layer": round(total_tok / total_s),
-            "sample": f"{seqs} of {len(ctx)} sequences of one layer ({total_tok} cached tokens), "
-                      f"fp64 C oracle, single thread, {total_s:.1f} s"}
+    res = {"value": round(total_kv / total_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "seq_tokens_per_s_per_layer": round(total_tok / total_s),
+           "sample": f"{seqs} whole sequence(s) of one layer of the {workload} workload ({total_tok} cached "
+                     f"tokens), fp64 C oracle, single thread, {total_s:.1f} s"}
+    return (res, step_secs) if per_step else res
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on this host, same workload, metric and unit.
-    Each step is a bounded sample: a few whole sequences of one layer."""
+    """--impl reference: the CPU oracle on this host, same workload, metric and unit;
+    each step is a bounded sample (--ref-seqs whole sequences of one layer)."""
     rank, _, world = dist_env()
     if rank != 0:
         return
-    import oracle
-    cfg = WORKLOADS[args.workload]
-    B, H_q, H_kv, d, dt = cfg["B"], cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
-    tdt = wl.TORCH_DTYPE[dt]
-    oracle.build()
-    gen = wl.generator(431 + 3)
-    ctx = make_lens(args.workload, gen, B)
-    N = B * cfg["width"]
-    paging = wl.allocate(ctx, N, cfg["width"], gen)
-    per_step = max(1, args.ref_seqs)
-    need = sorted(set(range(min(B, per_step * (args.steps + args.warmup)))))
-    # only the blocks the sampled sequences reference are materialised on the host
-    gh = wl.generator(431 + 200)
-    k_host = torch.zeros(N, H_kv, 16, d, dtype=tdt)
-    v_host = torch.zeros_like(k_host)
-    for b in need:
-        nb = wl.ceil_div(int(ctx[b]), 16)
-        blk = paging.tables[b, :nb].long()
-        k_host[blk] = wl.normal((nb, H_kv, 16, d), tdt, gh)
-        v_host[blk] = wl.normal((nb, H_kv, 16, d), tdt, gh)
-    q = wl.normal((B, H_q, d), tdt, gh)
-    secs, kvs, toks = [], 0, 0
-    for s in range(args.warmup + args.steps):
-        ids = [(s * per_step + i) % B for i in range(per_step)]
-        sec, kv = oracle_decode_sample(k_host, v_host, dt, paging.tables, ctx, q, ids, H_q, d)
-        if s >= args.warmup:
-            secs.append(sec)
-            kvs += kv
-            toks += int(ctx[ids].sum())
-    total = sum(secs)
-    value = kvs / total / 1e9
-    sample = (f"{per_step} whole sequence(s) of one layer per step ({args.workload}), fp64 C oracle, "
-              f"single thread")
-    res = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+    cpu, secs = cpu_oracle(args.workload, per_step=max(1, args.ref_seqs), steps=args.steps, warmup=args.warmup)
+    res = {"metric": METRIC, "value": cpu["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 2), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-           "config": {"workload": args.workload, "description": cfg["desc"]},
-           "seq_tokens_per_s_per_layer": round(toks / total),
-           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                            "sample": sample},
-           "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+           "config": {"workload": args.workload, "description": WORKLOADS[args.workload]["desc"]},
+           "seq_tokens_per_s_per_layer": cpu["seq_tokens_per_s_per_layer"],
+           "cpu_baseline": cpu,
+           "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
 

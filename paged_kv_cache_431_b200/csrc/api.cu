@@ -90,13 +90,16 @@ int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtenso
     return PKV_OK;
 }
 
-// Split-K partition size: 512 tokens unless the batch is too small to fill the GPU
-// with one-warp CTAs, then down to 128.
-static int choose_partition(int B, int H_kv, int max_ctx, const pkv_decode_opts* o)
+// Split-K partition size: about 256 KiB of K + V per partition whatever the storage
+// dtype (512 tokens for bf16 at head_dim 128, 1024 for int8 / fp8, 2048 for int4), so the
+// partials stay near 1.6% of the bytes read; smaller (down to 128 tokens) when the batch
+// is too small to fill the GPU with one-warp CTAs.
+static int choose_partition(int B, int H_kv, int max_ctx, int row_bytes, const pkv_decode_opts* o)
 {
     if (o && o->partition_tokens > 0) return o->partition_tokens;
+    int P = 256 * 1024 / (2 * row_bytes);
+    P = P < 128 ? 128 : (P > 4096 ? 4096 : P);
     const long target = 4L * num_sms() * 8;
-    int P = 512;
     while (P > 128) {
         const long parts = (max_ctx + P - 1) / P;
         if ((long)B * H_kv * (parts > 0 ? parts : 1) >= target) break;
@@ -225,7 +228,7 @@ int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, int src_
 static int decode_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, const pkv_decode_opts* opts, int* P,
                                int* max_parts)
 {
-    *P = choose_partition(num_seqs, pool->d.num_kv_heads, max_ctx, opts);
+    *P = choose_partition(num_seqs, pool->d.num_kv_heads, max_ctx, pool->row_bytes, opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
     *max_parts = max_ctx > 0 ? (max_ctx + *P - 1) / *P : 1;
     return PKV_OK;

@@ -39,6 +39,7 @@ struct Mma16Cfg {
     static constexpr int STAGE = 2 * TILE;
     static constexpr int SMEM = STAGES * STAGE + 1024;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(STAGES * STAGE >= 16 * (D + 4) * 4, "the epilogue stages 16 O rows in the ring");
 };
 
 template <int D, bool BF16, int NHT, int STAGES>

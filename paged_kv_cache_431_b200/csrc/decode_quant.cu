@@ -32,8 +32,10 @@ struct QCfg {
     static constexpr int ROW = DT == PKV_INT4 ? D / 2 : D;     // bytes per token row
     static constexpr int TILE = 16 * ROW;                      // one (block, head) tile
     static constexpr int STAGE = 2 * TILE;                     // K and V
-    static constexpr int STAGES = DT == PKV_INT4 ? 8 : 6;
-    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static constexpr int STAGES = DT == PKV_INT4 ? 4 : 3;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int STAGING = 16 * (D + 4) * 4;           // epilogue: 16 O rows, fp32
+    static constexpr int BODY = RING > STAGING ? RING : STAGING;   // the epilogue reuses the ring
     static constexpr int SWZ = ROW == 128 ? 7 : ROW == 64 ? 3 : 1;   // TMA 128/64/32-byte swizzle
     static constexpr int KRUN = ROW / 4;                       // K bytes per lane per token
     static constexpr int VRUN = ROW / 8;                       // V bytes per lane per row
@@ -100,10 +102,20 @@ __device__ __forceinline__ uint32_t i8x2(uint32_t wx, uint32_t sel)
     return h2_sub(__byte_perm(wx, 0x64646464u, sel), 1152.f);
 }
 
-// int4 codes, already XORed with 0x8 per nibble (u = c + 8): nibble s of each 16-bit half.
+// int4 codes, already XORed with 0x8 per nibble (u = c + 8): nibble s (0..3) of each
+// 16-bit half -> fp16 pair.  Even nibbles: 0x640X is 1024 + u; odd nibbles stay in
+// place, 0x64X0 is 1024 + 16 u, and one fused multiply-add by 1/16 removes both biases.
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, float m, float c)
+{
+    __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), __float2half2_rn(m), __float2half2_rn(c));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
 __device__ __forceinline__ uint32_t i4x2(uint32_t wx, int s)
 {
-    return h2_sub(((wx >> (4 * s)) & 0x000f000fu) | 0x64006400u, 1032.f);
+    const uint32_t w = (s & 2) ? (wx >> 8) : wx;
+    if (s & 1) return h2_fma((w & 0x00f000f0u) | 0x64006400u, 0.0625f, -72.f);
+    return h2_sub((w & 0x000f000fu) | 0x64006400u, 1032.f);
 }
 
 // e4m3 pair (low byte -> low half) -> fp16 pair.
@@ -193,8 +205,6 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     constexpr int ROW = Cfg::ROW, SWZ = Cfg::SWZ;
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[STAGES];
-    __shared__ int tbl[kMaxPartTiles];
-    __shared__ float2 tsc[kMaxPartTiles];   // (K scale, V scale) of each tile
 
     const int lane = threadIdx.x;
     const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -214,6 +224,11 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     const int ntok = min(p.part_tokens, ctx - tok0);
     const int ntiles = (ntok + kBlock - 1) / kBlock;
 
+    // dynamic shared memory: [K/V ring, reused by the epilogue][(K scale, V scale) per
+    // tile][block id per tile]
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    float2* tsc = reinterpret_cast<float2*>(smem + Cfg::BODY);
+    int* tbl = reinterpret_cast<int*>(tsc + p.part_tokens / kBlock);
     const int32_t* trow = p.tables + (size_t)b * p.W + tok0 / kBlock;
     for (int j = lane; j < ntiles; j += 32) {
         int blk = trow[j];
@@ -225,7 +240,6 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const size_t si = (size_t)blk * p.H_kv + g;
         tsc[j] = make_float2(p.k_scale[si], p.v_scale[si]);
     }
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     if (lane == 0) {
         for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
         mbar_fence_init();
@@ -381,10 +395,12 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 #pragma unroll
             for (int jj = 0; jj < MT_PER_WORD; ++jj) {
                 const int mt = k * MT_PER_WORD + jj;
-                va[jj][0] &= keep01;
-                va[jj][1] &= keep01;
-                va[jj][2] &= keep23;
-                va[jj][3] &= keep23;
+                if (nv < kBlock) {   // zero V of past-the-end tokens
+                    va[jj][0] &= keep01;
+                    va[jj][1] &= keep01;
+                    va[jj][2] &= keep23;
+                    va[jj][3] &= keep23;
+                }
 #pragma unroll
                 for (int hn = 0; hn < NHT; ++hn) {
                     mma16816<false>(o[mt][hn], va[jj], bh[hn][0], bh[hn][1]);
@@ -456,7 +472,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 template <int DT, int D>
 int launch_q(const DecodeParams& p, int nht, dim3 grid, cudaStream_t s, const CUtensorMap* tmk, const CUtensorMap* tmv)
 {
-    constexpr int smem = QCfg<DT, D>::SMEM;
+    const int smem = QCfg<DT, D>::BODY + 1024 + (p.part_tokens / kBlock) * (int)(sizeof(float2) + sizeof(int));
     auto k1 = decode_mmaq_kernel<DT, D, 1>;
     auto k2 = decode_mmaq_kernel<DT, D, 2>;
     auto kern = nht == 1 ? k1 : k2;
