@@ -33,7 +33,7 @@ int num_sms()
     return n;
 }
 
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+PFN_encode tensor_map_encoder()
 {
     static std::once_flag once;
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -51,7 +51,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 // boxes of 16 rows x (at most) 128 bytes with the matching shared-memory swizzle.
 static bool make_map(CUtensorMap* map, void* base, const pkv_pool_desc& d, int row_bytes)
 {
-    auto enc = encode_fn();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     const bool b16 = d.kv_dtype == PKV_F16 || d.kv_dtype == PKV_BF16;
     const int esize = b16 ? 2 : 1;
@@ -348,6 +348,12 @@ int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, int q_dt
     a.scale = scale;
     a.out = out;
     a.status = d.device_status;
+    if (prefill_tc_supported(a.d, a.G, a.kv_dtype)) {
+        CUtensorMap tmq;
+        auto enc = tensor_map_encoder();
+        if (!enc || !make_q_map(&tmq, q, chunk_len, num_q_heads, a.G, enc)) return PKV_ERR_CUDA;
+        return launch_prefill_tc(a, &tmq, tmk, tmv, static_cast<cudaStream_t>(stream));
+    }
     return launch_prefill(a, tmk, tmv, static_cast<cudaStream_t>(stream));
 }
 

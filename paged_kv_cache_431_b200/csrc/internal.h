@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -79,5 +80,14 @@ struct PrefillArgs {
 };
 
 int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
+
+using PFN_encode = PFN_cuTensorMapEncodeTiled_v12000;
+PFN_encode tensor_map_encoder();   // null when no driver is present
+
+// tcgen05 / TMEM form of the chunked prefill (prefill_tc.cu)
+bool prefill_tc_supported(int d, int G, int kv_dtype);
+bool make_q_map(CUtensorMap* map, const void* q, int C, int H_q, int G, PFN_encode enc);
+int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                      cudaStream_t s);
 
 }  // namespace pkv

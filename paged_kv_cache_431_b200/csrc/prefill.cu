@@ -87,24 +87,26 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         const uint32_t bar = smem_u32(&bars[s]);
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        // all four table entries first, so their loads overlap
+        int rows[4];
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
             const int lb = t * 4 + kb;        // logical block of the sequence
             // past the sequence's last block: load block 0 (in bounds); those keys are
             // masked and their V zeroed below
-            int row = g * kBlock;
-            if (lb < nblk_seq) {
-                int blk = p.table[lb];
-                if ((unsigned)blk >= (unsigned)p.N) {
-                    flag_status(p.status, PKV_DEV_BAD_BLOCK);
-                    blk = 0;
-                }
-                row = (blk * p.H_kv + g) * kBlock;
+            int blk = lb < nblk_seq ? p.table[lb] : 0;
+            if ((unsigned)blk >= (unsigned)p.N) {
+                flag_status(p.status, PKV_DEV_BAD_BLOCK);
+                blk = 0;
             }
+            rows[kb] = (blk * p.H_kv + g) * kBlock;
+        }
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
 #pragma unroll
             for (int x = 0; x < Cfg::NBOX; ++x) {
-                tma_load_2d(kdst + kb * Cfg::TILE + x * 2048, &tmK, x * 64, row, bar);
-                tma_load_2d(kdst + Cfg::KBYTES + kb * Cfg::TILE + x * 2048, &tmV, x * 64, row, bar);
+                tma_load_2d(kdst + kb * Cfg::TILE + x * 2048, &tmK, x * 64, rows[kb], bar);
+                tma_load_2d(kdst + Cfg::KBYTES + kb * Cfg::TILE + x * 2048, &tmV, x * 64, rows[kb], bar);
             }
         }
     };

@@ -1,0 +1,492 @@
+// prefill_tc.cu -- paged_prefill_chunk_attn on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Inference guide a2-inf-2, section "Chunked prefill", and "KV cache, continuous
+// batching and paged attention", section "Scheduling prefill and decode": a prompt
+// chunk of C positions P0 .. P0+C-1 attends causally to the paged context (possibly a
+// shared prefix, section "Prefix caching") and to itself.
+//
+// One CTA owns 128 query rows of one KV group -- 128/G positions x its G heads -- and
+// walks the keys in tiles of 128 (8 paged blocks):
+//   warp 0      TMA producer: Q once (a 3-D box over [position][head][dim]), then the
+//               K and V tiles of each step block by block through the pool's tensor
+//               maps into a 2-stage ring (128-byte swizzle, no multicast);
+//   warp 1      allocates 512 TMEM columns and issues the MMAs from one thread:
+//               S_t = Q . K_t^T into one of two TMEM score buffers (M=128, N=128, K=16
+//               per instruction), then O += P_{t-1} . V_{t-1} into the TMEM output
+//               accumulator, so the score MMA of a tile overlaps the softmax of the
+//               previous one;
+//   warps 2..5  softmax, one thread per query row (= TMEM lane): read the score row
+//               from TMEM, mask (causal bound P0 + position, end of sequence), keep the
+//               running max lazily (it moves only when the new max exceeds the old by 2^8,
+//               and then O is rescaled in TMEM), write P as a high and a low bf16/f16 part
+//               into shared memory (two MMAs keep P . V at ~16 mantissa bits), and finally
+//               read O, divide by the row sum and store fp32 rows.
+// Every wait is bounded; a timeout sets PKV_DEV_TIMEOUT and the CTA winds down.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pkv {
+
+namespace {
+
+constexpr int kD = 128;             // head dim handled here
+constexpr int kBM = 128;            // query rows per CTA
+constexpr int kBN = 128;            // keys per tile
+constexpr int kNS = 2;              // K/V ring stages
+constexpr int kQBytes = kBM * kD * 2;            // 32 KiB
+constexpr int kKVBytes = kBN * kD * 2;           // 32 KiB each for K and V
+constexpr int kPBytes = kBM * kBN * 2;           // 32 KiB each for P hi and P lo
+constexpr int kSmem = kQBytes + kNS * 2 * kKVBytes + 2 * kPBytes + 1024;
+constexpr uint32_t kTmemCols = 512;              // S0, S1, O (128 columns each)
+constexpr int kThreads = 192;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleSlack = 8.f;             // log2 units
+
+struct TcParams {
+    const int32_t* table;
+    float* out;
+    int32_t* status;
+    int P0, C, H_q, H_kv, G, N;
+    float scale_log2;
+};
+
+// ---- tcgen05 wrappers ------------------------------------------------------
+
+__device__ __forceinline__ uint64_t sdesc_k128(uint32_t addr)
+{
+    // K-major, 128-byte swizzle: rows of 128 B, 8-row atoms 1024 B apart (SBO), LBO unused (16 B)
+    return (uint64_t)((addr >> 4) & 0x3fff) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ uint64_t sdesc_mn128(uint32_t addr, uint32_t lbo_bytes)
+{
+    // MN-major, 128-byte swizzle: 64-element MN groups lbo_bytes apart (LBO), 8-row K groups
+    // 1024 B apart (SBO)
+    return (uint64_t)((addr >> 4) & 0x3fff) | ((uint64_t)((lbo_bytes >> 4) & 0x3fff) << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major, int M, int N)
+{
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// Wait with a bound; on timeout record it and raise the CTA's abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status)
+{
+    if (*abort_flag) return false;
+    if (mbar_wait_bounded(bar, parity)) return true;
+    *abort_flag = 1;
+    flag_status(status, PKV_DEV_TIMEOUT);
+    return false;
+}
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t kv_full[kNS];
+    uint64_t kv_empty[kNS];
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full;
+    uint64_t o_done;
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV)
+{
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ Bars bars;
+    __shared__ uint32_t s_tmem_base;
+    __shared__ volatile int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = blockIdx.y;
+    const int pos_per_cta = kBM / p.G;
+    const int i0 = blockIdx.x * pos_per_cta;                 // first chunk position of this CTA
+    const int i_end = min(p.C, i0 + pos_per_cta);
+    const int seq_len = p.P0 + p.C;
+    const int kend = p.P0 + i_end;                           // exclusive key bound of the CTA's last row
+    const int ntiles = (kend + kBN - 1) / kBN;
+    const int nblk_seq = (seq_len + kBlock - 1) / kBlock;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const uint32_t sQ = smem_u32(smem);
+    const uint32_t sK = sQ + kQBytes;                        // kNS stages of K
+    const uint32_t sV = sK + kNS * kKVBytes;                 // kNS stages of V
+    const uint32_t sPh = sV + kNS * kKVBytes;
+    const uint32_t sPl = sPh + kPBytes;
+
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        mbar_init(smem_u32(&bars.q_full), 1);
+        for (int s = 0; s < kNS; ++s) {
+            mbar_init(smem_u32(&bars.kv_full[s]), 1);
+            mbar_init(smem_u32(&bars.kv_empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&bars.s_full[b]), 1);
+            mbar_init(smem_u32(&bars.s_free[b]), 4);
+        }
+        mbar_init(smem_u32(&bars.p_full), 4);
+        mbar_init(smem_u32(&bars.o_done), 1);
+        mbar_fence_init();
+    }
+    if (warp == 1) {   // TMEM: S0 [0,128), S1 [128,256), O [256,384)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        // The whole warp walks the tiles: its 32 lanes hold the block ids of the next 4
+        // tiles (one coalesced load per 4 tiles, fetched a chunk ahead), lane 0 issues the
+        // copies.  Reading the table one entry at a time between copies would put a global
+        // load latency in front of every block.
+        constexpr int kBlkPerTile = kBN / kBlock;            // 8
+        constexpr int kTilesPerChunk = 32 / kBlkPerTile;     // 4
+        auto table_entry = [&](int lb) -> int {             // physical block of logical block lb
+            if (lb >= nblk_seq) return -1;                   // past the sequence
+            int blk = p.table[lb];
+            if ((unsigned)blk >= (unsigned)p.N) {
+                flag_status(p.status, PKV_DEV_BAD_BLOCK);
+                blk = 0;
+            }
+            return blk;
+        };
+        const uint32_t qb = smem_u32(&bars.q_full);
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            mbar_arrive_expect_tx(qb, kQBytes);
+            tma_load_3d(sQ, &tmQ, 0, g * p.G, i0, qb);
+            tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * p.G, i0, qb);
+        }
+        int cur = table_entry(lane);                         // chunk 0
+        int nxt = table_entry(32 + lane);                    // chunk 1
+        int issued = 0;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % kNS;
+            if (t > 0 && t % kTilesPerChunk == 0) {
+                cur = nxt;
+                nxt = table_entry((t / kTilesPerChunk + 1) * 32 + lane);
+            }
+            bool go = true;
+            if (lane == 0 && t >= kNS)
+                go = wait_or_abort(smem_u32(&bars.kv_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
+            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
+            const uint32_t fb = smem_u32(&bars.kv_full[s]);
+            if (lane == 0) mbar_arrive_expect_tx(fb, 2 * kKVBytes);
+#pragma unroll
+            for (int kb = 0; kb < kBlkPerTile; ++kb) {
+                const int blk = __shfl_sync(0xffffffffu, cur, (t % kTilesPerChunk) * kBlkPerTile + kb);
+                // past the sequence: block 0 (in bounds; those keys are masked and their V zeroed)
+                const int row = ((blk < 0 ? 0 : blk) * p.H_kv + g) * kBlock;
+                if (lane == 0) {
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, row, fb);
+                        tma_load_2d(sV + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmV, 64 * x, row, fb);
+                    }
+                }
+            }
+            issued = t + 1;
+        }
+        // do not leave while copies into this CTA's shared memory may be in flight
+        if (lane == 0 && s_abort) {
+            for (int t = max(0, issued - kNS); t < issued; ++t)
+                mbar_wait_bounded(smem_u32(&bars.kv_full[t % kNS]), (t / kNS) & 1);
+            mbar_wait_bounded(qb, 0);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_f16(BF16, false, kBM, kBN);
+            const uint32_t id_pv = idesc_f16(BF16, true, kBM, kD);
+            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status);
+            for (int t = 0; ok && t <= ntiles; ++t) {
+                if (t < ntiles) {
+                    const int s = t % kNS, b = t & 1;
+                    if (!wait_or_abort(smem_u32(&bars.kv_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
+                    if (t >= 2 && !wait_or_abort(smem_u32(&bars.s_free[b]), ((t - 2) >> 1) & 1, &s_abort, p.status))
+                        break;
+                    tc_fence_after();
+                    const uint32_t kbase = sK + s * kKVBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32;
+                        umma(tmem + b * kBN, sdesc_k128(sQ + off), sdesc_k128(kbase + off), id_qk, ks > 0);
+                    }
+                    umma_commit(smem_u32(&bars.s_full[b]));
+                }
+                if (t >= 1) {
+                    const int u = t - 1, s = u % kNS;
+                    if (!wait_or_abort(smem_u32(&bars.p_full), u & 1, &s_abort, p.status)) break;
+                    tc_fence_after();
+                    const uint32_t vbase = sV + s * kKVBytes;
+#pragma unroll
+                    for (int ks = 0; ks < kBN / 16; ++ks) {
+                        const uint32_t poff = (ks >> 2) * (kPBytes / 2) + (ks & 3) * 32;
+                        const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBytes / 2);
+                        umma(tmem + 2 * kBN, sdesc_k128(sPh + poff), bv, id_pv, u > 0 || ks > 0);
+                        umma(tmem + 2 * kBN, sdesc_k128(sPl + poff), bv, id_pv, true);
+                    }
+                    umma_commit(smem_u32(&bars.o_done));
+                    umma_commit(smem_u32(&bars.kv_empty[s]));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int quarter = warp & 3;                        // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;                   // query row of this thread
+        const int pos = i0 + r / p.G;
+        const int kmax = p.P0 + min(pos, p.C - 1) + 1;       // keys < kmax are visible
+        const int kmin_cta = p.P0 + i0 + 1;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float sl = p.scale_log2;
+        float m_used = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            const int b = t & 1;
+            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[b]), (t >> 1) & 1, &s_abort, p.status))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float x[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(trow + b * kBN + 32 * c, *reinterpret_cast<float(*)[32]>(&x[32 * c]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[b]));
+
+            const int key0 = t * kBN;
+            const bool need_mask = key0 + kBN > kmin_cta;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kBN; ++j) {
+                float v = x[j] * sl;
+                if (need_mask && key0 + j >= kmax) v = -INFINITY;
+                x[j] = v;
+                mx = fmaxf(mx, v);
+            }
+            float m_new = m_used;
+            if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
+            const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
+
+            // P = 2^(x - m) as high + low 16-bit parts, computed before waiting for the
+            // previous P . V so the exponentials overlap the tensor cores
+            const float mref = m_new == -INFINITY ? 0.f : m_new;
+            float sum = 0.f;
+            uint32_t ph[kBN / 2], pl[kBN / 2];
+#pragma unroll
+            for (int e = 0; e < kBN / 2; ++e) {
+                const float p0 = ex2(x[2 * e] - mref), p1 = ex2(x[2 * e + 1] - mref);
+                ph[e] = pack2<BF16>(p0, p1);
+                const float2 back = unpack2<BF16>(ph[e]);
+                pl[e] = pack2<BF16>(p0 - back.x, p1 - back.y);
+                sum += p0 + p1;
+            }
+            if (t > 0) {   // P . V of the previous tile done: P buffers free, O settled
+                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (t - 1) & 1, &s_abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                    for (int c = 0; c < kD / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(trow + 2 * kBN + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(trow + 2 * kBN + 32 * c, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // K-major rows with the 128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int e0 = hf * 32 + c * 4;
+                    const uint32_t off = hf * (kPBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(ph[e0]),
+                                 "r"(ph[e0 + 1]), "r"(ph[e0 + 2]), "r"(ph[e0 + 3])
+                                 : "memory");
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(pl[e0]),
+                                 "r"(pl[e0 + 1]), "r"(pl[e0 + 2]), "r"(pl[e0 + 3])
+                                 : "memory");
+                }
+            }
+            l_run = l_run * alpha + sum;
+            m_used = m_new;
+            // keys past the end of the sequence: zero their V rows (P is 0 there, V may be stale)
+            if (t == ntiles - 1 && key0 + kBN > seq_len) {
+                const int s = t % kNS;
+                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.kv_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                const int first = seq_len - key0;
+                const int tid = threadIdx.x - 64;             // 0..127
+                for (int i = tid; i < 2 * (kBN - first) * 8; i += 128) {
+                    const int x16 = i & 7, rowi = (i >> 3) % (kBN - first), half = (i >> 3) / (kBN - first);
+                    const uint32_t a = sV + s * kKVBytes + half * (kKVBytes / 2) + (first + rowi) * 128 + x16 * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
+        }
+        if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (ntiles - 1) & 1, &s_abort, p.status))) {
+            tc_fence_after();
+            const bool valid = pos < p.C;
+            const float inv = 1.f / l_run;
+            float* orow = p.out + ((size_t)pos * p.H_q + g * p.G + (r % p.G)) * kD;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                float o[32];
+                tmem_ld32(trow + 2 * kBN + 32 * c, o);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(orow + 32 * c + i) =
+                            make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int d, int G, int kv_dtype)
+{
+    return d == kD && G >= 1 && G <= kBM && (kBM % G) == 0 && (kv_dtype == PKV_BF16 || kv_dtype == PKV_F16);
+}
+
+// Q viewed as [C][H_q][d] with boxes of 64 dims x G heads x 128/G positions.
+bool make_q_map(CUtensorMap* map, const void* q, int C, int H_q, int G, PFN_encode enc)
+{
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H_q, (cuuint64_t)C};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H_q * kD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(kBM / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtensorMap* tmk, const CUtensorMap* tmv,
+                      cudaStream_t s)
+{
+    TcParams p;
+    p.table = a.table;
+    p.out = a.out;
+    p.status = a.status;
+    p.P0 = a.P0;
+    p.C = a.C;
+    p.H_q = a.H_q;
+    p.H_kv = a.H_kv;
+    p.G = a.G;
+    p.N = a.N;
+    p.scale_log2 = a.scale * kLog2e;
+    auto kern = a.kv_dtype == PKV_BF16 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    const int pos_per_cta = kBM / a.G;
+    const dim3 grid((a.C + pos_per_cta - 1) / pos_per_cta, a.H_kv);
+    kern<<<grid, kThreads, kSmem, s>>>(p, *tmq, *tmk, *tmv);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace pkv

@@ -21,6 +21,8 @@ CASES = [
     (40, 100, 32, 2, 128, wl.BF16),    # G = 16
     (123, 70, 12, 4, 128, wl.F16),     # G = 3
     (300, 129, 64, 8, 128, wl.BF16),   # 70B head shape
+    (77, 200, 16, 4, 128, wl.F16),     # G = 4, fp16
+    (0, 300, 4, 4, 128, wl.BF16),      # MHA from an empty context: rows with 1..300 keys
 ]
 
 
