@@ -249,7 +249,8 @@ def build_decode(args, cfg, dev, rank):
             pkv.kv_append(pool, lp, k_new[l], v_new[l], slots, workspace=aws)
             if ev is not None:
                 ev[l][0].record(stream)
-            pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws)
+            pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws,
+                                  engine=args.engine)
             if ev is not None:
                 ev[l][1].record(stream)
 
@@ -292,7 +293,8 @@ def build_decode(args, cfg, dev, rank):
         for l in range(L):
             stream.wait_event(ready[l])
             pkv.kv_append(pool, l % L_phys, dk[l], dv[l], dslots, workspace=aws)
-            pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, scale, max_ctx, out=dout[l], workspace=ws)
+            pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, scale, max_ctx, out=dout[l], workspace=ws,
+                                  engine=args.engine)
             e = torch.cuda.Event()
             e.record(stream)
             done.append(e)
@@ -312,7 +314,9 @@ def build_decode(args, cfg, dev, rank):
                 "kv_heads": H_kv, "head_dim": d, "kv_dtype": DTYPE_NAME[dt], "sum_ctx": int(ctx.sum()),
                 "physical_layer_pools": L_phys, "parallelism": "replicas",
                 "l2": f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V",
-                "partition_tokens": "auto"},
+                "partition_tokens": "auto",
+                "decode_engine": {0: "tensor cores (mma.sync)", 1: "tensor cores (mma.sync)",
+                                  2: "CUDA cores, packed fp32x2 FMA", 3: "CUDA cores, fp32 FMA"}[args.engine]},
         kv_bytes_per_step=kv * L, seq_tokens_per_step=int(ctx.sum()) * L, layers=L,
         roofline=dict(bound="hbm", kernel="paged_decode_attn (main + split-K merge)", alg_bytes=alg,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
@@ -603,6 +607,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--engine", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="decode engine: 0/1 tensor cores, 2 CUDA-core packed FMA, 3 CUDA-core FMA")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -146,7 +146,10 @@ PKV_API int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, 
 
 /* Tuning options for paged_decode_attn (NULL = defaults). */
 typedef struct {
-    int32_t engine;            /* 0 auto (tensor cores), 1 tensor-core mma, 2 CUDA-core FMA (16-bit pools) */
+    int32_t engine;            /* 0 auto (= 1); 1 tensor cores (warp-level mma.sync), every pool dtype;
+                                  2 CUDA-core FP32 FMA with packed fp32x2 pairs, 3 CUDA-core scalar FP32 FMA:
+                                  16-bit pools, head_dim 128, G 4 or 8, q 16-byte aligned (else
+                                  PKV_ERR_UNSUPPORTED); kept to measure the FP32-pipe form of the decode */
     int32_t partition_tokens;  /* tokens per split-K partition; 0 = chosen from the workload; else a
                                   multiple of 16 in [64, 16384] */
 } pkv_decode_opts;

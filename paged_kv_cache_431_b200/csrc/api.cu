@@ -263,7 +263,7 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     if (!is_quantized(d.kv_dtype) && q_dtype != d.kv_dtype) return PKV_ERR_DTYPE;
     if ((reinterpret_cast<uintptr_t>(q) & 3) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
     int engine = opts ? opts->engine : 0;
-    if (engine < 0 || engine > 2) return PKV_ERR_ARG;
+    if (engine < 0 || engine > 3) return PKV_ERR_ARG;
     if (engine == 0) engine = 1;
     int P, parts;
     int rc = decode_partitioning(pool, num_seqs, max_context_len, opts, &P, &parts);

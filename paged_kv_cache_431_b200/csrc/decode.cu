@@ -403,7 +403,11 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     const dim3 grid(a.max_parts, a.H_kv, a.B);
     const int nht = a.G <= 8 ? 1 : 2;
     int rc = PKV_ERR_UNSUPPORTED;
-    if (a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) {
+    if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && (a.engine == 2 || a.engine == 3)) {
+        if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
+            return PKV_ERR_UNSUPPORTED;
+        rc = launch_decode_simt(p, a.kv_dtype, a.G, a.engine == 2, grid, s, tmk, tmv);
+    } else if (a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) {
         if (a.engine != 1) return PKV_ERR_UNSUPPORTED;
         const bool bf = a.kv_dtype == PKV_BF16;
         if (a.d == 128) rc = bf ? launch_mma16<128, true>(p, nht, grid, s, tmk, tmv)

@@ -44,6 +44,11 @@ __device__ __forceinline__ uint32_t swz128(uint32_t tile, int t, int c)
 }
 
 
+// CUDA-core (FP32 FMA) decode for 16-bit pools (decode_simt.cu); f2 = packed fp32x2 FMA.
+bool decode_simt_supported(int d, int G, int kv_dtype);
+int launch_decode_simt(const DecodeParams& p, int kv_dtype, int G, bool f2, dim3 grid, cudaStream_t s,
+                       const CUtensorMap* tmk, const CUtensorMap* tmv);
+
 // Launch the quantized-pool decode kernel (decode_quant.cu).
 int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,
                         const CUtensorMap* tmk, const CUtensorMap* tmv);

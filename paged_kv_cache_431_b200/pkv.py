@@ -18,7 +18,7 @@ BLOCK_SIZE = 16
 F16, BF16, INT8, INT4, FP8E4M3 = 0, 1, 2, 3, 4
 QUANTIZED = (INT8, INT4, FP8E4M3)
 DEV_BAD_BLOCK, DEV_BAD_SLOT, DEV_BAD_LENGTH, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
-ENGINE_AUTO, ENGINE_MMA, ENGINE_FMA = 0, 1, 2
+ENGINE_AUTO, ENGINE_MMA, ENGINE_FMA2, ENGINE_FMA = 0, 1, 2, 3
 
 _TORCH16 = {F16: torch.float16, BF16: torch.bfloat16}
 

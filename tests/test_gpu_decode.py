@@ -237,3 +237,19 @@ def test_gqa70b_config_one_layer():
     assert pkv.read_device_status(pool) == 0
     seq_ids = torch.randperm(B, generator=g)[:8].tolist()
     assert _sampled_parity(pool, k_pool, v_pool, wl.BF16, q, paging.tables, ctx, out, d ** -0.5, seq_ids) <= TOL
+
+
+@pytest.mark.parametrize("engine", [pkv.ENGINE_FMA2, pkv.ENGINE_FMA], ids=["fma2", "fma"])
+@pytest.mark.parametrize("G,dtype", [(8, wl.BF16), (4, wl.F16)])
+def test_cuda_core_engines(engine, G, dtype):
+    """The CUDA-core (FP32 FMA) decode engines against the oracle, with split-K."""
+    g = wl.generator(1200 + G + engine)
+    H_kv = 4
+    lens = [1, 15, 16, 17, 100, 777, 1500] + torch.randint(1, 600, (3,), generator=g).tolist()
+    N = sum(wl.ceil_div(n, 16) for n in lens) + 3
+    wk = wl.decode_workload("fma", lens, H_kv * G, H_kv, 128, dtype, N, 100, 1300 + G)
+    pool = gpu_pool_from(wk)
+    ref = oracle_decode(wk)
+    for part in (0, 256):
+        out = run_decode(wk, pool, engine=engine, partition_tokens=part)
+        assert max_abs_diff(out, ref) <= TOL
