@@ -237,8 +237,8 @@ def build_decode(args, cfg, dev, rank):
     k_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     v_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     out = torch.empty(L, B, H_q, d, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx), 16), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition), 16),
+                     dtype=torch.uint8, device=dev)
     aws = torch.empty(max(pkv.kv_append_workspace_bytes(pool, B), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     scale = d ** -0.5
@@ -250,7 +250,7 @@ def build_decode(args, cfg, dev, rank):
             if ev is not None:
                 ev[l][0].record(stream)
             pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws,
-                                  engine=args.engine)
+                                  engine=args.engine, partition_tokens=args.partition)
             if ev is not None:
                 ev[l][1].record(stream)
 
@@ -294,7 +294,7 @@ def build_decode(args, cfg, dev, rank):
             stream.wait_event(ready[l])
             pkv.kv_append(pool, l % L_phys, dk[l], dv[l], dslots, workspace=aws)
             pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, scale, max_ctx, out=dout[l], workspace=ws,
-                                  engine=args.engine)
+                                  engine=args.engine, partition_tokens=args.partition)
             e = torch.cuda.Event()
             e.record(stream)
             done.append(e)
@@ -314,7 +314,7 @@ def build_decode(args, cfg, dev, rank):
                 "kv_heads": H_kv, "head_dim": d, "kv_dtype": DTYPE_NAME[dt], "sum_ctx": int(ctx.sum()),
                 "physical_layer_pools": L_phys, "parallelism": "replicas",
                 "l2": f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V",
-                "partition_tokens": "auto",
+                "partition_tokens": args.partition or "auto",
                 "decode_engine": {0: "tensor cores (mma.sync)", 1: "tensor cores (mma.sync)",
                                   2: "CUDA cores, packed fp32x2 FMA", 3: "CUDA cores, fp32 FMA"}[args.engine]},
         kv_bytes_per_step=kv * L, seq_tokens_per_step=int(ctx.sum()) * L, layers=L,
@@ -607,6 +607,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--partition", type=int, default=0,
+                    help="split-K partition size in tokens (0: chosen by the library)")
     ap.add_argument("--engine", type=int, default=0, choices=[0, 1, 2, 3],
                     help="decode engine: 0/1 tensor cores, 2 CUDA-core packed FMA, 3 CUDA-core FMA")
     args = ap.parse_args()

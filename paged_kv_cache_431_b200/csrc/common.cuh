@@ -84,6 +84,22 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------- programmatic dependent launch --
+
+// Let the next kernel on the stream (launched with programmatic stream serialization)
+// be scheduled before this grid finishes; it still waits for this grid's results.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grid this one depends on has completed and its writes are visible
+// (returns at once when the kernel was launched without that dependency).
+__device__ __forceinline__ void pdl_wait_primary()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------- TMA --
 
 // 2-D tiled bulk tensor load global -> shared, completion counted on `bar` (bytes).

@@ -52,6 +52,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     __shared__ __align__(8) uint64_t bars[STAGES];
     __shared__ int tbl[kMaxPartTiles];
 
+    pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
     const int lane = threadIdx.x;
     const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int r = lane >> 2, qd = lane & 3;
@@ -311,6 +312,7 @@ template <int D>
 __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
 {
     const int h = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
+    pdl_wait_primary();   // the partials of the decode kernel before this one
     const int ctx = checked_ctx(p, b, false);
     const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
     if (nparts <= 1) return;
@@ -420,10 +422,20 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     }
     if (rc != PKV_OK) return rc;
     if (a.max_parts > 1) {
-        const dim3 rgrid(a.H_q, a.B);
-        if (a.d == 128) decode_reduce_kernel<128><<<rgrid, 32, 0, s>>>(p);
-        else decode_reduce_kernel<64><<<rgrid, 32, 0, s>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return PKV_ERR_CUDA;
+        // programmatic dependent launch: scheduled while the decode grid's last wave runs
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.H_q, a.B);
+        cfg.blockDim = dim3(32);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = a.d == 128 ? cudaLaunchKernelEx(&cfg, decode_reduce_kernel<128>, p)
+                                         : cudaLaunchKernelEx(&cfg, decode_reduce_kernel<64>, p);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
     }
     return PKV_OK;
 }

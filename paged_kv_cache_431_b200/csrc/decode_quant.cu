@@ -206,6 +206,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[STAGES];
 
+    pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
     const int lane = threadIdx.x;
     const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int r = lane >> 2, qd = lane & 3;

@@ -67,6 +67,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     __shared__ __align__(16) float p_s[G][32];   // P of the tile, each value twice
     __shared__ float a_s[G], m_s[G], l_s[G];
 
+    pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
     const int lane = threadIdx.x;
     const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int dg = lane & 15, tg = lane >> 4;

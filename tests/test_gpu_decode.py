@@ -253,3 +253,26 @@ def test_cuda_core_engines(engine, G, dtype):
     for part in (0, 256):
         out = run_decode(wk, pool, engine=engine, partition_tokens=part)
         assert max_abs_diff(out, ref) <= TOL
+
+
+def test_workspace_reuse_across_shapes():
+    """One workspace, never cleared by the caller, serves a series of split-K calls of
+    different shapes in stream order (each call clears its own counters)."""
+    g = wl.generator(1400)
+    H_q, H_kv, d = 32, 8, 128
+    cases = []
+    for i, B in enumerate((7, 20, 3)):
+        lens = torch.randint(200, 2000, (B,), generator=g).tolist()
+        N = sum(wl.ceil_div(n, 16) for n in lens) + 2
+        cases.append(wl.decode_workload(f"reuse{i}", lens, H_q, H_kv, d, wl.BF16, N, 130, 1410 + i))
+    need = max(pkv.paged_decode_workspace_bytes(gpu_pool_from(wk), wk.B, H_q, 2000, partition_tokens=128)
+               for wk in cases)
+    ws = torch.full((need,), 0x5A, dtype=torch.uint8, device=DEV)   # stale contents
+    for rep in range(2):
+        for wk in cases:
+            pool = gpu_pool_from(wk)
+            out = pkv.paged_decode_attn(pool, 0, wk.q.to(DEV), wk.paging.tables.to(DEV), wk.paging.ctx_lens.to(DEV),
+                                        wk.scale, 2000, workspace=ws, partition_tokens=128)
+            torch.cuda.synchronize()
+            assert pkv.read_device_status(pool) == 0
+            assert max_abs_diff(out, oracle_decode(wk)) <= TOL
