@@ -15,7 +15,8 @@
 //               per instruction), then O += P_{t-1} . V_{t-1} into the TMEM output
 //               accumulator, so the score MMA of a tile overlaps the softmax of the
 //               previous one;
-//   warps 2..5  softmax, one thread per query row (= TMEM lane): read the score row
+//   warps 2..9  softmax, two threads per query row (= TMEM lane), each with half the
+//               keys of a tile and half the output dims: read the score row
 //               from TMEM, mask (causal bound P0 + position, end of sequence), keep the
 //               running max lazily (it moves only when the new max exceeds the old by 2^8,
 //               and then O is rescaled in TMEM), write P as a high and a low bf16/f16 part
@@ -38,7 +39,7 @@ constexpr int kKVBytes = kBN * kD * 2;           // 32 KiB each for K and V
 constexpr int kPBytes = kBM * kBN * 2;           // 32 KiB each for P hi and P lo
 constexpr int kSmem = kQBytes + kNS * 2 * kKVBytes + 2 * kPBytes + 1024;
 constexpr uint32_t kTmemCols = 512;              // S0, S1, O (128 columns each)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                    // producer, MMA, 8 softmax warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.f;             // log2 units
 
@@ -125,6 +126,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         : "memory");
 }
 
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr)
+{
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -155,6 +168,7 @@ struct Bars {
     uint64_t s_free[2];
     uint64_t p_full;
     uint64_t o_done;
+    uint64_t pair[4];          // the two softmax warps of a TMEM lane quarter
 };
 
 template <bool BF16>
@@ -193,9 +207,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&bars.s_full[b]), 1);
-            mbar_init(smem_u32(&bars.s_free[b]), 4);
+            mbar_init(smem_u32(&bars.s_free[b]), 8);
         }
-        mbar_init(smem_u32(&bars.p_full), 4);
+        mbar_init(smem_u32(&bars.p_full), 8);
+        for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars.pair[q]), 2);
         mbar_init(smem_u32(&bars.o_done), 1);
         mbar_fence_init();
     }
@@ -312,15 +327,42 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         }
     } else {
         // ------------------------------------------------------------ softmax
-        const int quarter = warp & 3;                        // TMEM lanes 32*quarter .. +31
+        // Warps 2..9.  quarter = warp % 4 fixes the 32 TMEM lanes (query rows) a warp may
+        // read; the two warps of a quarter split every row: hc = 0 takes keys 0-63 of a tile
+        // and output dims 0-63, hc = 1 the upper halves.  They combine their row maxima (and,
+        // at the end, their row sums) through spare TMEM columns, ordered by a 2-arrival
+        // mbarrier per quarter.
+        const int quarter = warp & 3;
+        const int hc = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;                   // query row of this thread
         const int pos = i0 + r / p.G;
         const int kmax = p.P0 + min(pos, p.C - 1) + 1;       // keys < kmax are visible
         const int kmin_cta = p.P0 + i0 + 1;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t xcol = trow + 3 * kBN;                // exchange columns 384..387
+        const uint32_t pair_bar = smem_u32(&bars.pair[quarter]);
         const float sl = p.scale_log2;
-        float m_used = -INFINITY, l_run = 0.f;
+        const bool pos_scale = sl > 0.f;
+        const float slx = pos_scale ? sl : 1.f;              // scale applied inside the exponent
+        float m_used = -INFINITY, l_half = 0.f;
         bool ok = true;
+        // exchange one value per row with the other warp of the quarter; `phase` counts uses
+        auto exchange = [&](float mine, int phase) -> float {
+            const uint32_t slot = xcol + (phase & 1) * 2;
+            tmem_st1(slot + hc, mine);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar);
+            if (!__all_sync(0xffffffffu, wait_or_abort(pair_bar, phase & 1, &s_abort, p.status))) {
+                ok = false;
+                return mine;
+            }
+            tc_fence_after();
+            const float other = tmem_ld1(slot + (hc ^ 1));
+            tmem_wait_ld();
+            return other;
+        };
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
             if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[b]), (t >> 1) & 1, &s_abort, p.status))) {
@@ -328,39 +370,56 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 break;
             }
             tc_fence_after();
-            float x[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(trow + b * kBN + 32 * c, *reinterpret_cast<float(*)[32]>(&x[32 * c]));
+            float x[kBN / 2];
+            tmem_ld32(trow + b * kBN + (kBN / 2) * hc, *reinterpret_cast<float(*)[32]>(&x[0]));
+            tmem_ld32(trow + b * kBN + (kBN / 2) * hc + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[b]));
 
-            const int key0 = t * kBN;
-            const bool need_mask = key0 + kBN > kmin_cta;
+            const int key0 = t * kBN + (kBN / 2) * hc;
+            const bool need_mask = t * kBN + kBN > kmin_cta;
             float mx = -INFINITY;
+            if (pos_scale) {        // max of the raw scores, scaled once
 #pragma unroll
-            for (int j = 0; j < kBN; ++j) {
-                float v = x[j] * sl;
-                if (need_mask && key0 + j >= kmax) v = -INFINITY;
-                x[j] = v;
-                mx = fmaxf(mx, v);
+                for (int j = 0; j < kBN / 2; ++j) {
+                    if (need_mask && key0 + j >= kmax) x[j] = -INFINITY;
+                    mx = fmaxf(mx, x[j]);
+                }
+                mx *= sl;
+            } else {
+#pragma unroll
+                for (int j = 0; j < kBN / 2; ++j) {
+                    x[j] = (need_mask && key0 + j >= kmax) ? -INFINITY : x[j] * sl;
+                    mx = fmaxf(mx, x[j]);
+                }
             }
+            mx = fmaxf(mx, exchange(mx, t));
+            if (!ok) break;
             float m_new = m_used;
             if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
             const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
 
-            // P = 2^(x - m) as high + low 16-bit parts, computed before waiting for the
-            // previous P . V so the exponentials overlap the tensor cores
+            // P = 2^(score - m) as high + low 16-bit parts, computed before waiting for the
+            // previous P . V so the exponentials overlap the tensor cores.  bf16: the high
+            // part is the truncation (upper half of the fp32 word), the low part the exact
+            // remainder rounded to bf16.
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             float sum = 0.f;
-            uint32_t ph[kBN / 2], pl[kBN / 2];
+            uint32_t ph[kBN / 4], pl[kBN / 4];
 #pragma unroll
-            for (int e = 0; e < kBN / 2; ++e) {
-                const float p0 = ex2(x[2 * e] - mref), p1 = ex2(x[2 * e + 1] - mref);
-                ph[e] = pack2<BF16>(p0, p1);
-                const float2 back = unpack2<BF16>(ph[e]);
-                pl[e] = pack2<BF16>(p0 - back.x, p1 - back.y);
+            for (int e = 0; e < kBN / 4; ++e) {
+                const float p0 = ex2(fmaf(x[2 * e], slx, -mref)), p1 = ex2(fmaf(x[2 * e + 1], slx, -mref));
+                if constexpr (BF16) {
+                    const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                    ph[e] = __byte_perm(u0, u1, 0x7632);
+                    pl[e] = pack2<true>(p0 - __uint_as_float(u0 & 0xffff0000u), p1 - __uint_as_float(u1 & 0xffff0000u));
+                } else {
+                    ph[e] = pack2<false>(p0, p1);
+                    const float2 back = unpack2<false>(ph[e]);
+                    pl[e] = pack2<false>(p0 - back.x, p1 - back.y);
+                }
                 sum += p0 + p1;
             }
             if (t > 0) {   // P . V of the previous tile done: P buffers free, O settled
@@ -371,44 +430,41 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                    for (int c = 0; c < kD / 32; ++c) {
+                    for (int c = 0; c < kD / 64; ++c) {
                         float o[32];
-                        tmem_ld32(trow + 2 * kBN + 32 * c, o);
+                        const uint32_t oc = trow + 2 * kBN + (kD / 2) * hc + 32 * c;
+                        tmem_ld32(oc, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(trow + 2 * kBN + 32 * c, o);
+                        tmem_st32(oc, o);
                     }
                     tmem_wait_st();
                 }
             }
-            // K-major rows with the 128-byte swizzle: 16-byte chunk c of row r at c ^ (r % 8)
+            // this warp's 64 keys are box hc of P: K-major rows with the 128-byte swizzle
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int e0 = hf * 32 + c * 4;
-                    const uint32_t off = hf * (kPBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(ph[e0]),
-                                 "r"(ph[e0 + 1]), "r"(ph[e0 + 2]), "r"(ph[e0 + 3])
-                                 : "memory");
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(pl[e0]),
-                                 "r"(pl[e0 + 1]), "r"(pl[e0 + 2]), "r"(pl[e0 + 3])
-                                 : "memory");
-                }
+            for (int c = 0; c < 8; ++c) {
+                const uint32_t off = hc * (kPBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(ph[4 * c]),
+                             "r"(ph[4 * c + 1]), "r"(ph[4 * c + 2]), "r"(ph[4 * c + 3])
+                             : "memory");
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(pl[4 * c]),
+                             "r"(pl[4 * c + 1]), "r"(pl[4 * c + 2]), "r"(pl[4 * c + 3])
+                             : "memory");
             }
-            l_run = l_run * alpha + sum;
+            l_half = l_half * alpha + sum;
             m_used = m_new;
             // keys past the end of the sequence: zero their V rows (P is 0 there, V may be stale)
-            if (t == ntiles - 1 && key0 + kBN > seq_len) {
+            if (t == ntiles - 1 && t * kBN + kBN > seq_len) {
                 const int s = t % kNS;
                 if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.kv_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
                     ok = false;
                     break;
                 }
-                const int first = seq_len - key0;
-                const int tid = threadIdx.x - 64;             // 0..127
-                for (int i = tid; i < 2 * (kBN - first) * 8; i += 128) {
+                const int first = seq_len - t * kBN;
+                const int tid = threadIdx.x - 64;             // 0..255
+                for (int i = tid; i < 2 * (kBN - first) * 8; i += 256) {
                     const int x16 = i & 7, rowi = (i >> 3) % (kBN - first), half = (i >> 3) / (kBN - first);
                     const uint32_t a = sV + s * kKVBytes + half * (kKVBytes / 2) + (first + rowi) * 128 + x16 * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
@@ -419,15 +475,17 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
         }
+        float l_tot = l_half;
+        if (ok) l_tot += exchange(l_half, ntiles);
         if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (ntiles - 1) & 1, &s_abort, p.status))) {
             tc_fence_after();
             const bool valid = pos < p.C;
-            const float inv = 1.f / l_run;
-            float* orow = p.out + ((size_t)pos * p.H_q + g * p.G + (r % p.G)) * kD;
+            const float inv = 1.f / l_tot;
+            float* orow = p.out + ((size_t)pos * p.H_q + g * p.G + (r % p.G)) * kD + (kD / 2) * hc;
 #pragma unroll 1
-            for (int c = 0; c < kD / 32; ++c) {
+            for (int c = 0; c < kD / 64; ++c) {
                 float o[32];
-                tmem_ld32(trow + 2 * kBN + 32 * c, o);
+                tmem_ld32(trow + 2 * kBN + (kD / 2) * hc + 32 * c, o);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
