@@ -229,6 +229,42 @@ PKV_API int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, 
                              int ctx_before, int chunk_len, int num_q_heads, float scale,
                              float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * kv_copy_blocks -- copy-on-write at divergence ([KVB] "Paged attention": blocks shared
+ * copy-on-write by parallel samples, beam search and common prefixes; [KVG]
+ * "PagedAttention": sequences with a common prefix point at the same blocks, copy-on-write
+ * at divergence).  For j < num_pairs, physical block dst[j] becomes a copy of block src[j]
+ * in every layer: its K and V tiles of all KV heads and, for quantized pools, its scales.
+ *   src, dst [device]: int32 [num_pairs].  The dst ids must be distinct and none may
+ *   appear in src (overlapping pairs race; the result is then undefined).
+ * An id outside [0, num_blocks) skips its pair and sets PKV_DEV_BAD_BLOCK.
+ */
+PKV_API int kv_copy_blocks(pkv_pool_t pool, const int32_t* src, const int32_t* dst, int num_pairs, void* stream);
+
+/* Bytes one block takes in host memory when swapped out (all layers, K and V, scales):
+ *   num_layers * 2 * num_kv_heads * 16 * row_bytes  +  num_layers * 2 * num_kv_heads * 4 (quantized).
+ * Layout of one swapped block: [layer][K, V][num_kv_heads][16][row_bytes], then
+ * [layer][K, V][num_kv_heads] fp32 scales.  Returns 0 for a NULL pool. */
+PKV_API size_t kv_swap_bytes_per_block(pkv_pool_t pool);
+
+/*
+ * kv_swap_out / kv_swap_in -- preemption by swapping ([KVG] "The scheduler, and
+ * preemption": when the cache runs out of blocks, the newest sequence is evicted and its
+ * blocks are swapped to host memory, or dropped and recomputed, and brought back on
+ * resume).  kv_swap_out copies blocks[j] into host slot j; kv_swap_in copies host slot j
+ * into blocks[j].  A slot is kv_swap_bytes_per_block bytes, slots are consecutive.
+ *   blocks [device]: int32 [num_blocks_to_move].
+ *   host: page-locked host memory mapped into the device's address space (cudaHostAlloc
+ *   or cudaHostRegister; the runtime maps it on every system with unified addressing),
+ *   16-byte aligned, at least num_blocks_to_move * kv_swap_bytes_per_block bytes.
+ *   Anything else returns PKV_ERR_ARG.  One kernel moves every byte over the host link.
+ * The host buffer is read or written asynchronously: do not touch it until the stream
+ * has passed the call.  An id outside [0, num_blocks) skips that block and sets
+ * PKV_DEV_BAD_BLOCK.
+ */
+PKV_API int kv_swap_out(pkv_pool_t pool, const int32_t* blocks, int num_blocks_to_move, void* host, void* stream);
+PKV_API int kv_swap_in(pkv_pool_t pool, const int32_t* blocks, int num_blocks_to_move, const void* host, void* stream);
+
 /* Synchronize `stream`, read and clear the pool's device status word.  *status_out [host]
  * receives the PKV_DEV_* bits (0 if the pool has no status word).  Returns PKV_ERR_INDEX
  * or PKV_ERR_TIMEOUT if bits were set, PKV_OK otherwise. */

@@ -252,3 +252,55 @@ def paged_prefill_chunk(pool: Pool, q, q_dtype: int, block_table, ctx_before: in
                                          _ptr(bt), bt.shape[0], ctx_before, C, float(scale), _ptr(out)),
            "paged_prefill_chunk")
     return out
+
+
+# ------------------------------------------------------- whole-block moves --
+
+def copy_blocks(pools: list, src, dst) -> None:
+    """Copy-on-write at divergence ("KV cache, continuous batching and paged attention",
+    section "Paged attention"): in every layer's pool, block dst[j] takes the K and V
+    tiles of all heads and the scales of block src[j].  Pairs are applied in order."""
+    for s, t in zip(np.asarray(src).tolist(), np.asarray(dst).tolist()):
+        for p in pools:
+            p.k[t] = p.k[s]
+            p.v[t] = p.v[s]
+            p.k_scale[t] = p.k_scale[s]
+            p.v_scale[t] = p.v_scale[s]
+
+
+def swap_image(pools: list, blocks) -> np.ndarray:
+    """Host image of swapped-out blocks ("KV cache, GQA, paging and continuous batching",
+    section "The scheduler, and preemption": a preempted sequence's blocks go to host
+    memory).  One row of bytes per block: for each layer its K then V tiles of all heads,
+    then (quantized pools) for each layer its K then V scales as fp32."""
+    quant = pools[0].dtype in (INT8, INT4, FP8)
+    rows = []
+    for b in np.asarray(blocks).tolist():
+        parts = []
+        for p in pools:
+            parts += [p.k[b].reshape(-1), p.v[b].reshape(-1)]
+        if quant:
+            for p in pools:
+                parts += [p.k_scale[b].view(np.uint8), p.v_scale[b].view(np.uint8)]
+        rows.append(np.concatenate(parts))
+    width = sum(2 * p.k[0].size for p in pools) + (sum(2 * p.H_kv * 4 for p in pools) if quant else 0)
+    return np.stack(rows) if rows else np.zeros((0, width), np.uint8)
+
+
+def swap_restore(pools: list, blocks, image: np.ndarray) -> None:
+    """Inverse of swap_image: block blocks[j] takes row j of the image, in place."""
+    quant = pools[0].dtype in (INT8, INT4, FP8)
+    for j, b in enumerate(np.asarray(blocks).tolist()):
+        row, at = image[j], 0
+        for p in pools:
+            n = p.k[b].size
+            p.k[b] = row[at:at + n].reshape(p.k[b].shape)
+            p.v[b] = row[at + n:at + 2 * n].reshape(p.v[b].shape)
+            at += 2 * n
+        if quant:
+            for p in pools:
+                n = 4 * p.H_kv
+                p.k_scale[b] = row[at:at + n].copy().view(np.float32)
+                p.v_scale[b] = row[at + n:at + 2 * n].copy().view(np.float32)
+                at += 2 * n
+        assert at == row.size

@@ -1,4 +1,4 @@
-"""Build libpkv.so in-tree from csrc/*.cu with nvcc for sm_100a.
+"""Build libpkv.so in-tree from csrc/*.cu (nvcc, sm_100a) and csrc/*.cpp (host C++, g++).
 
     python -m paged_kv_cache_431_b200.build [--force]
 
@@ -36,9 +36,16 @@ def _nvcc() -> str:
     return path if os.path.exists(path) else "nvcc"
 
 
+CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-Wall", "-I", INCLUDE]
+
+
+def _sources() -> list[str]:
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
+
+
 def _deps() -> list[str]:
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
-                  glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "pkv.h")])
+    return sorted(_sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
+                  glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def _stale(target: str, deps: list[str]) -> bool:
@@ -49,23 +56,26 @@ def _stale(target: str, deps: list[str]) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    srcs = _sources()
     deps = _deps()
     if not force and not _stale(LIB, deps):
         return LIB
     os.makedirs(OBJ, exist_ok=True)
     nvcc = _nvcc()
-    headers = [d for d in deps if not d.endswith(".cu")]
+    headers = [d for d in deps if not d.endswith((".cu", ".cpp"))]
 
     def compile_one(src: str) -> str:
         obj = os.path.join(OBJ, os.path.basename(src) + ".o")
         if force or _stale(obj, [src] + headers):
-            cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+            if src.endswith(".cpp"):
+                cmd = [os.environ.get("CXX", "g++"), *CXX_FLAGS, "-c", src, "-o", obj]
+            else:
+                cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
             if verbose:
                 print(" ".join(cmd), flush=True)
             res = subprocess.run(cmd, capture_output=True, text=True)
             if res.returncode != 0:
-                raise RuntimeError(f"nvcc failed on {src}:\n{res.stdout}\n{res.stderr}")
+                raise RuntimeError(f"compile failed on {src}:\n{res.stdout}\n{res.stderr}")
         return obj
 
     with ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:

@@ -8,6 +8,7 @@
 #include <new>
 
 #include "internal.h"
+#include "../../include/pkv_block_manager.h"
 
 namespace pkv {
 
@@ -131,6 +132,8 @@ const char* pkv_strerror(int status)
     case PKV_ERR_TIMEOUT: return "a kernel gave up waiting on a bulk copy";
     case PKV_ERR_INDEX: return "the device saw a block id, slot or context length out of range";
     case PKV_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case PKV_ERR_NO_BLOCKS: return "not enough free blocks in the pool";
+    case PKV_ERR_STATE: return "unknown, existing or swapped-out sequence, or a broken block-manager invariant";
     default: return "unknown status";
     }
 }

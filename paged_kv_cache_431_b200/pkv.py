@@ -81,6 +81,14 @@ def lib() -> ctypes.CDLL:
     L.paged_prefill_workspace_bytes.argtypes = [P, i32, i32, i32]
     L.paged_prefill_chunk_attn.restype = i32
     L.paged_prefill_chunk_attn.argtypes = [P, i32, P, i32, P, i32, i32, i32, i32, f32, P, P, sz, P]
+    L.kv_copy_blocks.restype = i32
+    L.kv_copy_blocks.argtypes = [P, P, P, i32, P]
+    L.kv_swap_bytes_per_block.restype = sz
+    L.kv_swap_bytes_per_block.argtypes = [P]
+    L.kv_swap_out.restype = i32
+    L.kv_swap_out.argtypes = [P, P, i32, P, P]
+    L.kv_swap_in.restype = i32
+    L.kv_swap_in.argtypes = [P, P, i32, P, P]
     L.pkv_read_device_status.restype = i32
     L.pkv_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     _lib = L
@@ -272,6 +280,43 @@ def paged_prefill_chunk_attn(pool: KVPool, layer: int, q: torch.Tensor, block_ta
     return out
 
 
+def kv_copy_blocks(pool: KVPool, src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    """Copy physical block src[j] onto block dst[j] (all layers, K, V and scales); int32 tensors."""
+    if src.shape != dst.shape or src.dim() != 1:
+        raise ValueError("src and dst must be int32 vectors of one length")
+    _check(lib().kv_copy_blocks(pool.handle, _ptr(src), _ptr(dst), src.shape[0], _stream(stream)),
+           "kv_copy_blocks")
+
+
+def kv_swap_bytes_per_block(pool: KVPool) -> int:
+    return int(lib().kv_swap_bytes_per_block(pool.handle))
+
+
+def _host_ptr(t: torch.Tensor):
+    if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+        raise ValueError("expected a contiguous pinned host tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_swap_buffer(pool: KVPool, blocks: torch.Tensor, host: torch.Tensor):
+    if host.numel() * host.element_size() < blocks.shape[0] * kv_swap_bytes_per_block(pool):
+        raise ValueError("host swap buffer too small")
+
+
+def kv_swap_out(pool: KVPool, blocks: torch.Tensor, host: torch.Tensor, stream=None) -> None:
+    """Copy blocks [int32, device] to consecutive slots of the pinned host buffer `host`."""
+    _check_swap_buffer(pool, blocks, host)
+    _check(lib().kv_swap_out(pool.handle, _ptr(blocks), blocks.shape[0], _host_ptr(host), _stream(stream)),
+           "kv_swap_out")
+
+
+def kv_swap_in(pool: KVPool, blocks: torch.Tensor, host: torch.Tensor, stream=None) -> None:
+    """Copy consecutive slots of the pinned host buffer `host` into blocks [int32, device]."""
+    _check_swap_buffer(pool, blocks, host)
+    _check(lib().kv_swap_in(pool.handle, _ptr(blocks), blocks.shape[0], _host_ptr(host), _stream(stream)),
+           "kv_swap_in")
+
+
 def read_device_status(pool: KVPool, stream=None) -> int:
     """Synchronize the stream and return (and clear) the pool's device status bits."""
     st = ctypes.c_int32(0)
@@ -279,3 +324,147 @@ def read_device_status(pool: KVPool, stream=None) -> int:
     if rc not in (0, -7, -8):
         _check(rc, "pkv_read_device_status")
     return int(st.value)
+
+
+# ------------------------------------------------------------ block manager --
+
+ERR_NO_BLOCKS, ERR_STATE = -10, -11
+
+
+class _BMStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("num_blocks", "free_blocks", "cached_blocks", "used_blocks",
+                                              "shared_blocks", "num_sequences", "prefix_queries", "prefix_hits",
+                                              "cow_copies", "evictions")]
+
+
+def _bm_lib():
+    L = lib()
+    if getattr(L, "_bm_ready", False):
+        return L
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    pi = ctypes.POINTER(ctypes.c_int32)
+    sig = {
+        "pkv_bm_create": (ctypes.c_int, [i32, ctypes.c_int, P]),
+        "pkv_bm_destroy": (ctypes.c_int, [P]),
+        "pkv_bm_free_blocks": (i64, [P]),
+        "pkv_bm_refcount": (ctypes.c_int, [P, i32]),
+        "pkv_bm_add_sequence": (ctypes.c_int, [P, i64, pi, i32, pi]),
+        "pkv_bm_blocks_needed": (ctypes.c_int, [P, i64, i32]),
+        "pkv_bm_append_slots": (ctypes.c_int, [P, i64, pi, i32, pi, pi, pi, pi]),
+        "pkv_bm_fork": (ctypes.c_int, [P, i64, i64]),
+        "pkv_bm_free_sequence": (ctypes.c_int, [P, i64]),
+        "pkv_bm_block_table": (ctypes.c_int, [P, i64, pi, i32, pi, pi]),
+        "pkv_bm_swap_out": (ctypes.c_int, [P, i64, pi, i32, pi]),
+        "pkv_bm_swap_in": (ctypes.c_int, [P, i64, pi, i32, pi]),
+        "pkv_bm_get_stats": (ctypes.c_int, [P, ctypes.POINTER(_BMStats)]),
+        "pkv_bm_check": (ctypes.c_int, [P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    L._bm_ready = True
+    return L
+
+
+def _i32_array(values):
+    values = list(values)
+    return (ctypes.c_int32 * max(1, len(values)))(*values)
+
+
+class BlockManager:
+    """Host-side block manager of a paged KV cache (free list, reference counts,
+    copy-on-write, prefix cache, swap bookkeeping); a thin wrapper of pkv_bm_* in libpkv.
+
+    Methods raise PkvError on a non-zero status; ``append_slots`` returns
+    ``(slot_mapping list, cow pair or None)``."""
+
+    def __init__(self, num_blocks: int, enable_prefix_cache: bool = True):
+        self._L = _bm_lib()
+        h = ctypes.c_void_p()
+        _check(self._L.pkv_bm_create(num_blocks, 1 if enable_prefix_cache else 0, ctypes.byref(h)), "pkv_bm_create")
+        self.handle = h
+        self.num_blocks = num_blocks
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            self._L.pkv_bm_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def free_blocks(self) -> int:
+        n = int(self._L.pkv_bm_free_blocks(self.handle))
+        _check(min(n, 0), "pkv_bm_free_blocks")
+        return n
+
+    def refcount(self, block: int) -> int:
+        n = self._L.pkv_bm_refcount(self.handle, block)
+        _check(min(n, 0), "pkv_bm_refcount")
+        return n
+
+    def add_sequence(self, seq_id: int, prompt=None, n_prompt: int | None = None) -> int:
+        """Register a sequence; returns the number of prompt tokens found in the prefix cache."""
+        toks = None if prompt is None else _i32_array(prompt)
+        n = len(prompt) if prompt is not None else int(n_prompt or 0)
+        cached = ctypes.c_int32(0)
+        _check(self._L.pkv_bm_add_sequence(self.handle, seq_id, toks, n, ctypes.byref(cached)),
+               "pkv_bm_add_sequence")
+        return int(cached.value)
+
+    def blocks_needed(self, seq_id: int, n: int) -> int:
+        r = self._L.pkv_bm_blocks_needed(self.handle, seq_id, n)
+        _check(min(r, 0), "pkv_bm_blocks_needed")
+        return r
+
+    def append_slots(self, seq_id: int, n: int, tokens=None):
+        slots = (ctypes.c_int32 * max(1, n))()
+        src, dst, ncow = ctypes.c_int32(-1), ctypes.c_int32(-1), ctypes.c_int32(0)
+        toks = None if tokens is None else _i32_array(tokens)
+        if tokens is not None and len(tokens) != n:
+            raise ValueError("len(tokens) != n")
+        _check(self._L.pkv_bm_append_slots(self.handle, seq_id, toks, n, slots, ctypes.byref(src), ctypes.byref(dst),
+                                           ctypes.byref(ncow)), "pkv_bm_append_slots")
+        return list(slots)[:n], ((int(src.value), int(dst.value)) if ncow.value else None)
+
+    def fork(self, parent_id: int, child_id: int) -> None:
+        _check(self._L.pkv_bm_fork(self.handle, parent_id, child_id), "pkv_bm_fork")
+
+    def free_sequence(self, seq_id: int) -> None:
+        _check(self._L.pkv_bm_free_sequence(self.handle, seq_id), "pkv_bm_free_sequence")
+
+    def block_table(self, seq_id: int):
+        """(list of physical blocks, number of tokens)."""
+        nb, nt = ctypes.c_int32(0), ctypes.c_int32(0)
+        rc = self._L.pkv_bm_block_table(self.handle, seq_id, None, 0, ctypes.byref(nb), ctypes.byref(nt))
+        if rc not in (0, -2):
+            _check(rc, "pkv_bm_block_table")
+        buf = (ctypes.c_int32 * max(1, nb.value))()
+        _check(self._L.pkv_bm_block_table(self.handle, seq_id, buf, nb.value, None, None), "pkv_bm_block_table")
+        return list(buf)[:nb.value], int(nt.value)
+
+    def swap_out(self, seq_id: int):
+        """Release the sequence's blocks; returns them (to be copied out with kv_swap_out)."""
+        table, _ = self.block_table(seq_id)
+        buf = (ctypes.c_int32 * max(1, len(table)))()
+        n = ctypes.c_int32(0)
+        _check(self._L.pkv_bm_swap_out(self.handle, seq_id, buf, len(table), ctypes.byref(n)), "pkv_bm_swap_out")
+        return list(buf)[:n.value]
+
+    def swap_in(self, seq_id: int, num_blocks: int):
+        """Give a swapped-out sequence fresh blocks; returns them (to be filled with kv_swap_in)."""
+        buf = (ctypes.c_int32 * max(1, num_blocks))()
+        n = ctypes.c_int32(0)
+        _check(self._L.pkv_bm_swap_in(self.handle, seq_id, buf, num_blocks, ctypes.byref(n)), "pkv_bm_swap_in")
+        return list(buf)[:n.value]
+
+    def stats(self) -> dict:
+        s = _BMStats()
+        _check(self._L.pkv_bm_get_stats(self.handle, ctypes.byref(s)), "pkv_bm_get_stats")
+        return {n: int(getattr(s, n)) for n, _ in _BMStats._fields_}
+
+    def check(self) -> None:
+        _check(self._L.pkv_bm_check(self.handle), "pkv_bm_check")

@@ -14,15 +14,20 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
-    return re.findall(r"^PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, re.M)
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, re.M)
+    return names
 
 
 def test_header_declares_the_entry_points():
     names = set(declared_functions())
-    for n in ("kv_pool_create", "kv_append", "paged_decode_attn", "paged_prefill_chunk_attn"):
+    for n in ("kv_pool_create", "kv_append", "paged_decode_attn", "paged_prefill_chunk_attn", "kv_copy_blocks",
+              "kv_swap_out", "kv_swap_in", "pkv_bm_create", "pkv_bm_append_slots", "pkv_bm_check"):
         assert n in names
-    assert len(names) >= 12
+    assert len(names) >= 30
 
 
 def test_library_exports_every_declared_symbol():
@@ -119,5 +124,41 @@ def test_quantized_append_needs_bf16_source_and_workspace():
         assert L.kv_append(h, 0, fake, fake, pkv.F16, fake, 10, fake, need, None) == -3
         assert L.kv_append(h, 0, fake, fake, pkv.BF16, fake, 10, None, 0, None) == -5
         assert L.kv_append(h, 0, fake, fake, pkv.BF16, fake, 10, fake, need - 4, None) == -5
+    finally:
+        L.kv_pool_destroy(h)
+
+
+@pytest.mark.parametrize("dtype,row", [(pkv.BF16, 256), (pkv.INT8, 128), (pkv.INT4, 64), (pkv.FP8E4M3, 128)])
+def test_swap_slot_size_is_one_block_of_every_layer(dtype, row):
+    """A swapped block holds, for each layer, K and V of every KV head (16 rows each) and,
+    quantized, one fp32 scale per (K/V, head)."""
+    L = pkv.lib()
+    quant = dtype in pkv.QUANTIZED
+    rc, h = _create(num_layers=3, num_kv_heads=8, head_dim=128, kv_dtype=dtype,
+                    k_scale=0x30000 if quant else None, v_scale=0x40000 if quant else None)
+    assert rc == 0
+    try:
+        assert L.kv_swap_bytes_per_block(h) == 3 * 2 * 8 * 16 * row + (3 * 2 * 8 * 4 if quant else 0)
+    finally:
+        L.kv_pool_destroy(h)
+    assert L.kv_swap_bytes_per_block(None) == 0
+
+
+def test_block_moves_validate_on_the_host():
+    L = pkv.lib()
+    rc, h = _create()
+    fake = ctypes.c_void_p(0x50000)
+    try:
+        assert L.kv_copy_blocks(None, fake, fake, 1, None) == -1
+        assert L.kv_copy_blocks(h, fake, fake, -1, None) == -2
+        assert L.kv_copy_blocks(h, None, None, 0, None) == 0
+        assert L.kv_copy_blocks(h, None, fake, 2, None) == -1
+        assert L.kv_swap_out(h, fake, -1, fake, None) == -2
+        assert L.kv_swap_out(h, None, 0, None, None) == 0
+        assert L.kv_swap_in(h, fake, 1, None, None) == -1
+        # pageable (not page-locked) or misaligned host memory is refused
+        buf = ctypes.create_string_buffer(1 << 16)
+        assert L.kv_swap_out(h, fake, 1, ctypes.cast(buf, ctypes.c_void_p), None) == -2
+        assert L.kv_swap_in(h, fake, 1, ctypes.c_void_p(ctypes.addressof(buf) + 8), None) == -2
     finally:
         L.kv_pool_destroy(h)

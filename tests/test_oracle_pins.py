@@ -483,3 +483,67 @@ def test_quant_block_reuse_starts_fresh(dtype):
     # ...but a write that does not start the block keeps (and may only grow) the scale
     oracle.kv_append(pool, small[:1], small[:1], oracle.BF16, np.array([3], np.int32))
     assert pool.k_scale[0, 0] >= np.float32(amax) / np.float32(Q)
+
+
+def _random_layers(L, N, H, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    pools = []
+    for _ in range(L):
+        p = oracle.Pool(N, H, d, dtype)
+        p.k[...] = rng.integers(0, 256, p.k.shape, dtype=np.uint8)
+        p.v[...] = rng.integers(0, 256, p.v.shape, dtype=np.uint8)
+        if dtype == oracle.FP8:
+            p.k[(p.k & 0x7F) == 0x7F] = 0x7E
+            p.v[(p.v & 0x7F) == 0x7F] = 0x7E
+        p.k_scale[...] = rng.random(p.k_scale.shape, dtype=np.float32) * 0.05
+        p.v_scale[...] = rng.random(p.v_scale.shape, dtype=np.float32) * 0.05
+        pools.append(p)
+    return pools
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.INT8, oracle.INT4, oracle.FP8])
+def test_copied_block_reads_like_its_source(dtype):
+    """Copy-on-write ("Paged attention" on the continuous-batching page): after copying a
+    sequence's blocks to fresh ids, attention through the new table equals attention
+    through the old one in every layer, and blocks outside the pairs are untouched."""
+    L, N, H, d = 2, 24, 2, 64
+    pools = _random_layers(L, N, H, d, dtype, 11 + dtype)
+    if dtype == oracle.F16:   # finite halves only
+        for p in pools:
+            p.k[...] = (np.random.default_rng(1).standard_normal(p.k.shape[:-1] + (d,)).astype(np.float16)
+                        .view(np.uint8))
+            p.v[...] = (np.random.default_rng(2).standard_normal(p.v.shape[:-1] + (d,)).astype(np.float16)
+                        .view(np.uint8))
+    before = [p.copy() for p in pools]
+    old, new = [3, 17, 5], [20, 1, 9]
+    oracle.copy_blocks(pools, old, new)
+    q = f16_bits(np.random.default_rng(3).standard_normal((1, 4, d)))
+    for l, p in enumerate(pools):
+        a = oracle.paged_decode(p, q, oracle.F16, np.array([old]), np.array([40]), 0.125)
+        b = oracle.paged_decode(p, q, oracle.F16, np.array([new]), np.array([40]), 0.125)
+        np.testing.assert_array_equal(a, b)
+        keep = [i for i in range(N) if i not in new]
+        assert np.array_equal(p.k[keep], before[l].k[keep]) and np.array_equal(p.v[keep], before[l].v[keep])
+        assert np.array_equal(p.k_scale[keep], before[l].k_scale[keep])
+
+
+@pytest.mark.parametrize("dtype,row", [(oracle.BF16, 128), (oracle.INT8, 64), (oracle.INT4, 32), (oracle.FP8, 64)])
+def test_swap_image_size_and_round_trip(dtype, row):
+    """Swapping ("The scheduler, and preemption" on the GQA page): a block's host image is
+    all of its layers' K and V tiles (and scales), L * 2 * H * 16 * row_bytes (+ L * 2 * H * 4)
+    bytes; restoring the image into other blocks reproduces the pool contents there."""
+    L, N, H, d = 3, 20, 2, 64
+    pools = _random_layers(L, N, H, d, dtype, 40 + dtype)
+    quant = dtype in (oracle.INT8, oracle.INT4, oracle.FP8)
+    img = oracle.swap_image(pools, [4, 11])
+    assert img.shape == (2, L * 2 * H * 16 * row + (L * 2 * H * 4 if quant else 0))
+    # the first tile in the image is layer 0's K tile of head 0 of block 4
+    assert np.array_equal(img[0, :16 * row], pools[0].k[4, 0].reshape(-1))
+    target = [p.copy() for p in pools]
+    oracle.swap_restore(target, [0, 19], img)
+    for p, t in zip(pools, target):
+        for s, dd in ((4, 0), (11, 19)):
+            assert np.array_equal(t.k[dd], p.k[s]) and np.array_equal(t.v[dd], p.v[s])
+            if quant:
+                assert np.array_equal(t.k_scale[dd], p.k_scale[s]) and np.array_equal(t.v_scale[dd], p.v_scale[s])
+    assert oracle.swap_image(pools, []).shape == (0, img.shape[1])
