@@ -359,16 +359,26 @@ def build_prefix_chunk(args, cfg, dev, rank):
     v_chunk = wl.normal((C, H_kv, d), torch.bfloat16, gd, dev)
     out_dec = torch.empty(B, H_q, d, dtype=torch.float32, device=dev)
     out_chunk = torch.empty(C, H_q, d, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx), 16), dtype=torch.uint8,
-                     device=dev)
+    cascade = args.decode_form == "cascade"
+    if cascade:
+        ws_bytes = pkv.paged_decode_cascade_workspace_bytes(pool, B, H_q, max_ctx, P0)
+    else:
+        ws_bytes = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     scale = d ** -0.5
+
+    def decode(q, out):
+        if cascade:   # the 4,000-token shared prompt once per KV group on the tensor cores
+            pkv.paged_decode_attn_cascade(pool, 0, q, tables, ctx_d, scale, max_ctx, P0, out=out, workspace=ws)
+        else:
+            pkv.paged_decode_attn(pool, 0, q, tables, ctx_d, scale, max_ctx, out=out, workspace=ws)
 
     def step(ev=None):
         pkv.kv_append(pool, 0, k_dec, v_dec, dec_slots)
         if ev is not None:
             ev[0][0].record(stream)
-        pkv.paged_decode_attn(pool, 0, q_dec, tables, ctx_d, scale, max_ctx, out=out_dec, workspace=ws)
+        decode(q_dec, out_dec)
         if ev is not None:
             ev[0][1].record(stream)
         pkv.kv_append(pool, 0, k_chunk, v_chunk, chunk_slots)
@@ -396,7 +406,7 @@ def build_prefix_chunk(args, cfg, dev, rank):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         pkv.kv_append(pool, 0, dk[:B], dv[:B], dec_slots)
-        pkv.paged_decode_attn(pool, 0, dq[:B], tables, ctx_d, scale, max_ctx, out=dout[:B], workspace=ws)
+        decode(dq[:B], dout[:B])
         pkv.kv_append(pool, 0, dk[B:], dv[B:], chunk_slots)
         pkv.paged_prefill_chunk_attn(pool, 0, dq[B:], chunk_table, P0, scale, out=dout[B:])
         hout.copy_(dout, non_blocking=True)
@@ -408,6 +418,8 @@ def build_prefix_chunk(args, cfg, dev, rank):
                 "sum_ctx_decode": int(ctx.sum()), "unique_kv_blocks": unique_blocks,
                 "unique_kv_bytes": unique_blocks * H_kv * 16 * d * 2 * 2,
                 "chunk_gflop": round(flops / 1e9, 2), "parallelism": "replicas",
+                "decode_form": ("cascade: the shared prefix once per KV group on tensor cores + per-sequence "
+                                "suffix split-K + merge") if cascade else "plain split-K decode",
                 "l2": "steady state, no flush: the shared prefix stays in L2 across the 256 decodes (as in real "
                       "prefix reuse)"},
         kv_bytes_per_step=dec_kv + chunk_kv, seq_tokens_per_step=int(ctx.sum()), layers=1,
@@ -416,7 +428,7 @@ def build_prefix_chunk(args, cfg, dev, rank):
                       peak_source=f"{kind} (MEASURED_PEAKS.json bf16_tflops, burst: a short kernel)",
                       traffic=kernel_traffic("prefill_prefix_chunk", PREFILL_SRCS), call_index=1,
                       decode_alg_bytes=dec_alg),
-        launches_per_step=4 + (1 if ws.numel() > 16 else 0), dtype="bf16",
+        launches_per_step=(6 if cascade else 4 + (1 if ws.numel() > 16 else 0)), dtype="bf16",
         h2d=sum(t.numel() * t.element_size() for t in (hq, hk, hv)), d2h=hout.numel() * 4, calls_per_step=2)
     return step, e2e_step, info, pool
 
@@ -609,6 +621,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition", type=int, default=0,
                     help="split-K partition size in tokens (0: chosen by the library)")
+    ap.add_argument("--decode-form", default="cascade", choices=["cascade", "plain"],
+                    help="prefix_chunk: decode the shared-prefix batch in the cascade form or plainly")
     ap.add_argument("--engine", type=int, default=0, choices=[0, 1, 2, 3],
                     help="decode engine: 0/1 tensor cores, 2 CUDA-core packed FMA, 3 CUDA-core FMA")
     args = ap.parse_args()

@@ -74,6 +74,7 @@ extern "C" {
 #define PKV_DEV_BAD_SLOT    0x2  /* slot_mapping entry >= num_blocks * 16               */
 #define PKV_DEV_BAD_LENGTH  0x4  /* context_len < 0, > 16 * table width, or > max_context_len */
 #define PKV_DEV_TIMEOUT     0x8  /* a bounded wait on a bulk copy ran out               */
+#define PKV_DEV_BAD_PREFIX  0x10 /* cascade decode: a table does not start with the shared prefix */
 
 typedef struct pkv_pool* pkv_pool_t;   /* opaque host-side handle */
 
@@ -208,6 +209,40 @@ PKV_API int paged_decode_attn_noalloc(pkv_pool_t pool, int layer, const void* q,
                                       const int32_t* context_lens, int num_seqs, int num_q_heads,
                                       int max_context_len, float scale, float* out,
                                       const pkv_decode_opts* opts, void* stream);
+
+/* Workspace paged_decode_attn_cascade needs (bytes): num_seqs * num_q_heads * (1 + suffix
+ * partitions) * (head_dim + 2) * 4.  0 for an unsupported shape.  With shared_prefix_len 0
+ * it equals paged_decode_workspace_bytes. */
+PKV_API size_t paged_decode_cascade_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads,
+                                                    int max_context_len, int shared_prefix_len,
+                                                    const pkv_decode_opts* opts);
+
+/*
+ * paged_decode_attn_cascade -- the decode of paged_decode_attn for a batch whose sequences
+ * all begin with the same shared_prefix_len tokens in the same physical blocks ([INF]
+ * "Prefix caching": requests attach to the cached blocks of a common prefix; [KVG] "Prefix
+ * caching": a 4,000-token system prompt shared by every request).  The result is the same
+ * attention over each sequence's whole context; it is computed in two parts merged with
+ * the log-sum-exp rule:
+ *   - the prefix once per KV group for the whole batch, as a dense tensor-core contraction
+ *     of all B * G query rows against the prefix keys (the blocks of block_tables row 0);
+ *   - each sequence's own tokens shared_prefix_len .. context_len-1 as in paged_decode_attn.
+ * Arguments as paged_decode_attn, plus:
+ *   shared_prefix_len: a multiple of 16, 0 < shared_prefix_len <= every context_len and
+ *     <= 16 * block_table_width; every table's first shared_prefix_len / 16 entries must
+ *     equal row 0's (the device checks and sets PKV_DEV_BAD_PREFIX otherwise; a context
+ *     shorter than the prefix sets PKV_DEV_BAD_LENGTH).  0 runs paged_decode_attn.
+ *   workspace [device]: paged_decode_cascade_workspace_bytes bytes, 16-byte aligned (always
+ *     required).  q [device] 16-byte aligned.
+ * Supported: 16-bit pools with head_dim 128 and 128 % G == 0 (PKV_ERR_UNSUPPORTED otherwise);
+ * q_dtype equal to the pool dtype.
+ */
+PKV_API int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_dtype,
+                                      const int32_t* block_tables, int block_table_width,
+                                      const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                      int max_context_len, int shared_prefix_len, float scale, float* out,
+                                      void* workspace, size_t workspace_bytes, const pkv_decode_opts* opts,
+                                      void* stream);
 
 /* Workspace paged_prefill_chunk_attn needs (bytes). */
 PKV_API size_t paged_prefill_workspace_bytes(pkv_pool_t pool, int chunk_len, int num_q_heads, int ctx_before);

@@ -103,6 +103,12 @@ def lib(path: str | None = None):
         _lib.orc_paged_prefill_chunk.restype = i32
         _lib.orc_paged_prefill_chunk.argtypes = [i32, i32, i32, i32, P, P, P, P, P, i32, i32, P, i32, i32,
                                                  i32, f32, P]
+        _lib.orc_paged_decode_window.restype = i32
+        _lib.orc_paged_decode_window.argtypes = [i32, i32, i32, i32, P, P, P, P, P, i32, i32, P, i32, P, i32, f32,
+                                                 i32, P]
+        _lib.orc_paged_prefill_chunk_window.restype = i32
+        _lib.orc_paged_prefill_chunk_window.argtypes = [i32, i32, i32, i32, P, P, P, P, P, i32, i32, P, i32, i32,
+                                                        i32, f32, i32, P]
     return _lib
 
 
@@ -226,30 +232,33 @@ def kv_append(pool: Pool, k_src, v_src, src_dtype: int, slots) -> None:
                                src_dtype, _ptr(slots), T), "kv_append")
 
 
-def paged_decode(pool: Pool, q, q_dtype: int, block_tables, ctx_lens, scale: float) -> np.ndarray:
-    """Decode attention, fp64 [B, H_q, d]."""
+def paged_decode(pool: Pool, q, q_dtype: int, block_tables, ctx_lens, scale: float, window: int = 0) -> np.ndarray:
+    """Decode attention, fp64 [B, H_q, d]; window > 0: only the `window` most recent positions."""
     q = as_u16(q)
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     cl = np.ascontiguousarray(ctx_lens, dtype=np.int32)
     B, H_q, d = q.shape
     assert d == pool.d and bt.shape[0] == B and cl.shape == (B,)
     out = np.empty((B, H_q, d), np.float64)
-    _check(lib().orc_paged_decode(pool.N, pool.H_kv, pool.d, pool.dtype, _ptr(pool.k), _ptr(pool.v),
-                                  _ptr(pool.k_scale), _ptr(pool.v_scale), _ptr(q), q_dtype, H_q,
-                                  _ptr(bt), bt.shape[1], _ptr(cl), B, float(scale), _ptr(out)),
+    _check(lib().orc_paged_decode_window(pool.N, pool.H_kv, pool.d, pool.dtype, _ptr(pool.k), _ptr(pool.v),
+                                         _ptr(pool.k_scale), _ptr(pool.v_scale), _ptr(q), q_dtype, H_q,
+                                         _ptr(bt), bt.shape[1], _ptr(cl), B, float(scale), int(window), _ptr(out)),
            "paged_decode")
     return out
 
 
-def paged_prefill_chunk(pool: Pool, q, q_dtype: int, block_table, ctx_before: int, scale: float) -> np.ndarray:
-    """Chunked-prefill attention of C query positions after ctx_before cached ones, fp64 [C, H_q, d]."""
+def paged_prefill_chunk(pool: Pool, q, q_dtype: int, block_table, ctx_before: int, scale: float,
+                        window: int = 0) -> np.ndarray:
+    """Chunked-prefill attention of C query positions after ctx_before cached ones, fp64 [C, H_q, d];
+    window > 0: each row sees only the `window` most recent positions up to itself."""
     q = as_u16(q)
     bt = np.ascontiguousarray(block_table, dtype=np.int32).reshape(-1)
     C, H_q, d = q.shape
     out = np.empty((C, H_q, d), np.float64)
-    _check(lib().orc_paged_prefill_chunk(pool.N, pool.H_kv, pool.d, pool.dtype, _ptr(pool.k), _ptr(pool.v),
-                                         _ptr(pool.k_scale), _ptr(pool.v_scale), _ptr(q), q_dtype, H_q,
-                                         _ptr(bt), bt.shape[0], ctx_before, C, float(scale), _ptr(out)),
+    _check(lib().orc_paged_prefill_chunk_window(pool.N, pool.H_kv, pool.d, pool.dtype, _ptr(pool.k),
+                                                _ptr(pool.v), _ptr(pool.k_scale), _ptr(pool.v_scale), _ptr(q),
+                                                q_dtype, H_q, _ptr(bt), bt.shape[0], ctx_before, C, float(scale),
+                                                int(window), _ptr(out)),
            "paged_prefill_chunk")
     return out
 

@@ -373,23 +373,24 @@ int orc_kv_append(int N, int H_kv, int d, int dtype,
 }
 
 /* ------------------------------------------------------------- attention --
- * Softmax attention of one query row over n keys gathered through a block table
+ * Softmax attention of one query row over keys lo .. n-1 gathered through a block table
  * ([KVG] "What it is": the cache holds K and V of every earlier token; [KVB] "Paged
  * attention": the attention kernel follows the block table).  In fp64:
  *   s_t = scale * sum_j q_j K[t][j];  m = max_t s_t;  w_t = exp(s_t - m);
- *   out_j = sum_t w_t V[t][j] / sum_t w_t;   n == 0 gives zeros.
+ *   out_j = sum_t w_t V[t][j] / sum_t w_t;   no keys give zeros.
+ * lo > 0 only for sliding-window attention (see window_start).
  */
 static int attend_one(int N, int H_kv, int d, int dtype,
                       const uint8_t* k_pool, const uint8_t* v_pool,
                       const float* k_scale, const float* v_scale,
-                      const double* qrow, int g, const int32_t* table, int W, int n,
+                      const double* qrow, int g, const int32_t* table, int W, int lo, int n,
                       double scale, double* s_buf, double* out)
 {
     for (int j = 0; j < d; ++j) out[j] = 0.0;
-    if (n <= 0) return ORC_OK;
+    if (n <= lo) return ORC_OK;
     if ((n + ORC_BLOCK - 1) / ORC_BLOCK > W) return ORC_ERR_ARG;
     double m = -INFINITY;
-    for (int t = 0; t < n; ++t) {
+    for (int t = lo; t < n; ++t) {
         int blk = table[t / ORC_BLOCK], off = t % ORC_BLOCK;
         if (blk < 0 || blk >= N) return ORC_ERR_INDEX;
         double acc = 0.0;
@@ -399,7 +400,7 @@ static int attend_one(int N, int H_kv, int d, int dtype,
         if (s_buf[t] > m) m = s_buf[t];
     }
     double denom = 0.0;
-    for (int t = 0; t < n; ++t) {
+    for (int t = lo; t < n; ++t) {
         int blk = table[t / ORC_BLOCK], off = t % ORC_BLOCK;
         double w = exp(s_buf[t] - m);
         denom += w;
@@ -413,6 +414,22 @@ static int attend_one(int N, int H_kv, int d, int dtype,
 /* Decode: one new query token per sequence attends to its whole cached context.
  * q is [B][H_q][d] (f16 or bf16), block_tables [B][W], ctx_lens [B], out [B][H_q][d].
  * [KVG] "Mechanics": GQA shares one KV head across G = H_q / H_kv query heads. */
+/* Sliding-window attention ([KVB] "The KV cache": sliding-window or hybrid local/global
+ * attention layers shrink what a query reads): a query at position pos sees the `window`
+ * most recent positions pos - window + 1 .. pos; window 0 means no window.  For a query
+ * whose keys end at n (exclusive), the first visible key is: */
+static int window_start(int n, int window)
+{
+    return (window > 0 && n > window) ? n - window : 0;
+}
+
+int orc_paged_decode_window(int N, int H_kv, int d, int dtype,
+                            const uint8_t* k_pool, const uint8_t* v_pool,
+                            const float* k_scale, const float* v_scale,
+                            const uint16_t* q, int q_dtype, int H_q,
+                            const int32_t* block_tables, int W, const int32_t* ctx_lens, int B,
+                            float scale, int window, double* out);
+
 int orc_paged_decode(int N, int H_kv, int d, int dtype,
                      const uint8_t* k_pool, const uint8_t* v_pool,
                      const float* k_scale, const float* v_scale,
@@ -420,6 +437,19 @@ int orc_paged_decode(int N, int H_kv, int d, int dtype,
                      const int32_t* block_tables, int W, const int32_t* ctx_lens, int B,
                      float scale, double* out)
 {
+    return orc_paged_decode_window(N, H_kv, d, dtype, k_pool, v_pool, k_scale, v_scale, q, q_dtype, H_q,
+                                   block_tables, W, ctx_lens, B, scale, 0, out);
+}
+
+/* Decode with an optional sliding window (window 0: the whole context). */
+int orc_paged_decode_window(int N, int H_kv, int d, int dtype,
+                            const uint8_t* k_pool, const uint8_t* v_pool,
+                            const float* k_scale, const float* v_scale,
+                            const uint16_t* q, int q_dtype, int H_q,
+                            const int32_t* block_tables, int W, const int32_t* ctx_lens, int B,
+                            float scale, int window, double* out)
+{
+    if (window < 0) return ORC_ERR_ARG;
     if (N <= 0 || H_kv <= 0 || d <= 0 || H_q <= 0 || B < 0 || W <= 0 || H_q % H_kv)
         return ORC_ERR_ARG;
     if (row_bytes(dtype, d) <= 0 || (q_dtype != ORC_F16 && q_dtype != ORC_BF16))
@@ -438,7 +468,8 @@ int orc_paged_decode(int N, int H_kv, int d, int dtype,
             size_t qo = ((size_t)b * H_q + h) * d;
             for (int j = 0; j < d; ++j) qrow[j] = src_value(q, q_dtype, qo + j);
             rc = attend_one(N, H_kv, d, dtype, k_pool, v_pool, k_scale, v_scale, qrow, h / G,
-                            block_tables + (size_t)b * W, W, ctx_lens[b], (double)scale, s_buf, out + qo);
+                            block_tables + (size_t)b * W, W, window_start(ctx_lens[b], window), ctx_lens[b],
+                            (double)scale, s_buf, out + qo);
         }
     free(s_buf); free(qrow);
     return rc;
@@ -449,6 +480,13 @@ int orc_paged_decode(int N, int H_kv, int d, int dtype,
  * in the pool.  Query row i attends causally to positions 0 .. P0+i, i.e. to the
  * earlier paged context and to its own chunk up to itself.
  * q is [C][H_q][d], block_table [W], out [C][H_q][d]. */
+int orc_paged_prefill_chunk_window(int N, int H_kv, int d, int dtype,
+                                   const uint8_t* k_pool, const uint8_t* v_pool,
+                                   const float* k_scale, const float* v_scale,
+                                   const uint16_t* q, int q_dtype, int H_q,
+                                   const int32_t* block_table, int W, int ctx_before, int C,
+                                   float scale, int window, double* out);
+
 int orc_paged_prefill_chunk(int N, int H_kv, int d, int dtype,
                             const uint8_t* k_pool, const uint8_t* v_pool,
                             const float* k_scale, const float* v_scale,
@@ -456,6 +494,20 @@ int orc_paged_prefill_chunk(int N, int H_kv, int d, int dtype,
                             const int32_t* block_table, int W, int ctx_before, int C,
                             float scale, double* out)
 {
+    return orc_paged_prefill_chunk_window(N, H_kv, d, dtype, k_pool, v_pool, k_scale, v_scale, q, q_dtype, H_q,
+                                          block_table, W, ctx_before, C, scale, 0, out);
+}
+
+/* Chunked prefill with an optional sliding window: row i sees positions
+ * max(0, ctx_before + i + 1 - window) .. ctx_before + i (window 0: all earlier ones). */
+int orc_paged_prefill_chunk_window(int N, int H_kv, int d, int dtype,
+                                   const uint8_t* k_pool, const uint8_t* v_pool,
+                                   const float* k_scale, const float* v_scale,
+                                   const uint16_t* q, int q_dtype, int H_q,
+                                   const int32_t* block_table, int W, int ctx_before, int C,
+                                   float scale, int window, double* out)
+{
+    if (window < 0) return ORC_ERR_ARG;
     if (N <= 0 || H_kv <= 0 || d <= 0 || H_q <= 0 || C < 0 || ctx_before < 0 || W <= 0 || H_q % H_kv)
         return ORC_ERR_ARG;
     if (row_bytes(dtype, d) <= 0 || (q_dtype != ORC_F16 && q_dtype != ORC_BF16))
@@ -470,7 +522,8 @@ int orc_paged_prefill_chunk(int N, int H_kv, int d, int dtype,
             size_t qo = ((size_t)i * H_q + h) * d;
             for (int j = 0; j < d; ++j) qrow[j] = src_value(q, q_dtype, qo + j);
             rc = attend_one(N, H_kv, d, dtype, k_pool, v_pool, k_scale, v_scale, qrow, h / G,
-                            block_table, W, ctx_before + i + 1, (double)scale, s_buf, out + qo);
+                            block_table, W, window_start(ctx_before + i + 1, window), ctx_before + i + 1,
+                            (double)scale, s_buf, out + qo);
         }
     free(s_buf); free(qrow);
     return rc;

@@ -305,6 +305,135 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     return launch_decode(a, tmk, tmv, static_cast<cudaStream_t>(stream));
 }
 
+// ---- shared-prefix (cascade) decode ------------------------------------------------
+
+static bool cascade_shape_ok(pkv_pool_t pool, int num_q_heads, int max_context_len, int prefix_len)
+{
+    const pkv_pool_desc& d = pool->d;
+    if (num_q_heads <= 0 || num_q_heads % d.num_kv_heads) return false;
+    const int G = num_q_heads / d.num_kv_heads;
+    return prefill_tc_supported(d.head_dim, G, d.kv_dtype) && prefix_len > 0 && prefix_len % PKV_BLOCK_SIZE == 0 &&
+           max_context_len >= prefix_len;
+}
+
+static int cascade_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, int prefix_len,
+                                const pkv_decode_opts* opts, int* P, int* suffix_parts)
+{
+    const int rest = max_ctx - prefix_len;
+    *P = choose_partition(num_seqs, pool->d.num_kv_heads, rest > 0 ? rest : 1, pool->row_bytes, opts);
+    if (!valid_partition(*P)) return PKV_ERR_ARG;
+    *suffix_parts = rest > 0 ? (rest + *P - 1) / *P : 1;
+    return PKV_OK;
+}
+
+size_t paged_decode_cascade_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_context_len,
+                                            int shared_prefix_len, const pkv_decode_opts* opts)
+{
+    if (!pool || num_seqs < 0 || max_context_len < 0 || shared_prefix_len < 0) return 0;
+    if (shared_prefix_len == 0) return paged_decode_workspace_bytes(pool, num_seqs, num_q_heads, max_context_len, opts);
+    if (!cascade_shape_ok(pool, num_q_heads, max_context_len, shared_prefix_len)) return 0;
+    int P, parts;
+    if (cascade_partitioning(pool, num_seqs, max_context_len, shared_prefix_len, opts, &P, &parts) != PKV_OK) return 0;
+    return (size_t)num_seqs * num_q_heads * (1 + parts) * (pool->d.head_dim + 2) * sizeof(float);
+}
+
+int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_dtype, const int32_t* block_tables,
+                              int block_table_width, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                              int max_context_len, int shared_prefix_len, float scale, float* out, void* workspace,
+                              size_t workspace_bytes, const pkv_decode_opts* opts, void* stream)
+{
+    if (!pool) return PKV_ERR_NULL;
+    if (shared_prefix_len < 0) return PKV_ERR_ARG;
+    if (shared_prefix_len == 0)
+        return paged_decode_attn(pool, layer, q, q_dtype, block_tables, block_table_width, context_lens, num_seqs,
+                                 num_q_heads, max_context_len, scale, out, workspace, workspace_bytes, opts, stream);
+    const pkv_pool_desc& d = pool->d;
+    if (layer < 0 || layer >= d.num_layers || num_seqs < 0 || num_q_heads <= 0 || block_table_width <= 0 ||
+        max_context_len < 0 || num_seqs > 65535)
+        return PKV_ERR_ARG;
+    if (num_q_heads % d.num_kv_heads) return PKV_ERR_SHAPE;
+    if (shared_prefix_len % PKV_BLOCK_SIZE || max_context_len < shared_prefix_len ||
+        (long long)block_table_width * PKV_BLOCK_SIZE < shared_prefix_len)
+        return PKV_ERR_SHAPE;
+    if (!cascade_shape_ok(pool, num_q_heads, max_context_len, shared_prefix_len)) return PKV_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !block_tables || !context_lens || !out) return PKV_ERR_NULL;
+    if (q_dtype != d.kv_dtype) return PKV_ERR_DTYPE;
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
+    int engine = opts ? opts->engine : 0;
+    if (engine < 0 || engine > 3) return PKV_ERR_ARG;
+    if (engine == 0) engine = 1;
+    int P, parts;
+    int rc = cascade_partitioning(pool, num_seqs, max_context_len, shared_prefix_len, opts, &P, &parts);
+    if (rc != PKV_OK) return rc;
+    const int slots = 1 + parts;
+    const size_t need = (size_t)num_seqs * num_q_heads * slots * (d.head_dim + 2) * sizeof(float);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15)) return PKV_ERR_WORKSPACE;
+    const CUtensorMap *tmk = nullptr, *tmv = nullptr;
+    rc = layer_maps(pool, layer, &tmk, &tmv);
+    if (rc != PKV_OK) return rc;
+    float* ws_o = static_cast<float*>(workspace);
+    float* ws_ml = ws_o + (size_t)num_seqs * num_q_heads * slots * d.head_dim;
+    const int G = num_q_heads / d.num_kv_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // 1. the shared prefix, once per KV group for the whole batch, on the tensor cores:
+    //    rows = (sequence, head of the group), keys = the prefix blocks of table row 0
+    PrefillArgs pa;
+    pa.q = q;
+    pa.q_dtype = q_dtype;
+    pa.table = block_tables;
+    pa.W = shared_prefix_len / PKV_BLOCK_SIZE;
+    pa.P0 = 0;
+    pa.C = num_seqs;
+    pa.H_q = num_q_heads;
+    pa.H_kv = d.num_kv_heads;
+    pa.G = G;
+    pa.N = d.num_blocks;
+    pa.d = d.head_dim;
+    pa.kv_dtype = d.kv_dtype;
+    pa.scale = scale;
+    pa.out = nullptr;
+    pa.status = d.device_status;
+    pa.cascade_nkeys = shared_prefix_len;
+    pa.ws_slots = slots;
+    pa.ws_o = ws_o;
+    pa.ws_ml = ws_ml;
+    CUtensorMap tmq;
+    auto enc = tensor_map_encoder();
+    if (!enc || !make_q_map(&tmq, q, num_seqs, num_q_heads, G, enc)) return PKV_ERR_CUDA;
+    rc = launch_prefill_tc(pa, &tmq, tmk, tmv, s);
+    if (rc != PKV_OK) return rc;
+
+    // 2. each sequence's own suffix as split-K partitions into slots 1.., then the merge
+    DecodeArgs a;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.tables = block_tables;
+    a.W = block_table_width;
+    a.ctx_lens = context_lens;
+    a.B = num_seqs;
+    a.H_q = num_q_heads;
+    a.H_kv = d.num_kv_heads;
+    a.G = G;
+    a.N = d.num_blocks;
+    a.d = d.head_dim;
+    a.kv_dtype = d.kv_dtype;
+    a.part_tokens = P;
+    a.max_parts = parts;
+    a.scale = scale;
+    a.k_scale = nullptr;
+    a.v_scale = nullptr;
+    a.out = out;
+    a.ws_o = ws_o;
+    a.ws_ml = ws_ml;
+    a.status = d.device_status;
+    a.engine = engine;
+    a.tok_base = shared_prefix_len;
+    a.part_base = 1;
+    return launch_decode(a, tmk, tmv, s);
+}
+
 size_t paged_prefill_workspace_bytes(pkv_pool_t pool, int chunk_len, int num_q_heads, int ctx_before)
 {
     (void)pool;

@@ -59,10 +59,10 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int hbase = g * p.G;
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
-    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
-    const int tok0 = part * p.part_tokens;
+    const int nparts = part_count(p, ctx);
+    const int tok0 = p.tok_base + part * p.part_tokens;
     if (tok0 >= ctx) {
-        if (part == 0) {   // empty context: a zero row
+        if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
             for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
         }
@@ -254,7 +254,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     // ---- epilogue: O rows [head][dim] through shared memory, then coalesced stores
 #pragma unroll
     for (int hr = 0; hr < NHT; ++hr) l_run[hr] = warp_sum_quad(l_run[hr]);
-    const bool final_out = (nparts == 1);
+    const bool final_out = (p.part_base == 0 && nparts == 1);
     float* so = reinterpret_cast<float*>(smem);
     constexpr int SR = D + 4;   // padded row stride (floats)
     __syncwarp();
@@ -288,7 +288,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int i = lane; i < p.G * (D / 4); i += 32) {
             const int h = i / (D / 4), c4 = i % (D / 4);
             const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
-            *reinterpret_cast<float4*>(p.ws_o + ((row0 + h) * p.max_parts + part) * D + 4 * c4) = v;
+            *reinterpret_cast<float4*>(p.ws_o + ws_slot(p, row0 + h, part) * D + 4 * c4) = v;
         }
         if (qd == 0) {
 #pragma unroll
@@ -296,7 +296,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 const int h = r + 8 * hr;
                 if (h < p.G) {
                     float2 ml = make_float2(m_run[hr], l_run[hr]);
-                    *reinterpret_cast<float2*>(p.ws_ml + ((row0 + h) * p.max_parts + part) * 2) = ml;
+                    *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) = ml;
                 }
             }
         }
@@ -306,7 +306,8 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 // ---------------------------------------------------------------------------
 // Split-K merge: out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
 // One warp per (query head, sequence); sequences that fit one partition were written
-// directly by the main kernel and are skipped.
+// directly by the main kernel and are skipped.  In the shared-prefix (cascade) form slot 0
+// holds the prefix's partial and the suffix partitions follow.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
@@ -314,9 +315,14 @@ __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
     const int h = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
     pdl_wait_primary();   // the partials of the decode kernel before this one
     const int ctx = checked_ctx(p, b, false);
-    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
-    if (nparts <= 1) return;
-    const size_t base = ((size_t)b * p.H_q + h) * p.max_parts;
+    if (p.prefix_blocks > 0 && h == 0) {   // cascade: every table must start with row 0's prefix
+        bool same = true;
+        for (int j = lane; j < p.prefix_blocks; j += 32) same &= p.tables[(size_t)b * p.W + j] == p.tables[j];
+        if (!__all_sync(0xffffffffu, same) && lane == 0) flag_status(p.status, PKV_DEV_BAD_PREFIX);
+    }
+    const int nparts = p.part_base + part_count(p, ctx);
+    if (p.part_base == 0 && nparts <= 1) return;
+    const size_t base = ((size_t)b * p.H_q + h) * p.slots;
     const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + base;
     float M = -INFINITY;
     for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
@@ -399,6 +405,10 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.N = a.N;
     p.part_tokens = a.part_tokens;
     p.max_parts = a.max_parts;
+    p.tok_base = a.tok_base;
+    p.part_base = a.part_base;
+    p.slots = a.part_base + a.max_parts;
+    p.prefix_blocks = a.part_base ? a.tok_base / kBlock : 0;
     p.q_bf16 = a.q_dtype == PKV_BF16;
     p.scale_log2 = a.scale * kLog2e;
 
@@ -421,7 +431,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         rc = launch_decode_quant(p, a.kv_dtype, a.d, nht, grid, s, tmk, tmv);
     }
     if (rc != PKV_OK) return rc;
-    if (a.max_parts > 1) {
+    if (a.max_parts > 1 || a.part_base > 0) {
         // programmatic dependent launch: scheduled while the decode grid's last wave runs
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(a.H_q, a.B);

@@ -20,6 +20,11 @@ struct DecodeParams {
     float* ws_ml;
     int32_t* status;
     int W, H_q, H_kv, G, N, part_tokens, max_parts;
+    // Partitions cover tokens tok_base .. ctx-1 and write workspace slots part_base + part of
+    // a row of `slots`.  Plain decode: 0, 0, max_parts.  Shared-prefix (cascade) decode:
+    // tok_base = prefix length, part_base = 1 (slot 0 holds the prefix's partial).
+    int tok_base, part_base, slots;
+    int prefix_blocks;      // cascade: table entries every sequence must share with row 0
     int q_bf16;             // q dtype: 1 bf16, 0 f16
     float scale_log2;
 };
@@ -28,12 +33,24 @@ struct DecodeParams {
 __device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool report)
 {
     int ctx = p.ctx_lens[b];
-    const int cap = min(p.W * kBlock, p.max_parts * p.part_tokens);
-    if (ctx < 0 || ctx > cap) {
+    const int cap = min(p.W * kBlock, p.tok_base + p.max_parts * p.part_tokens);
+    if (ctx < p.tok_base || ctx > cap) {
         if (report) flag_status(p.status, PKV_DEV_BAD_LENGTH);
-        ctx = ctx < 0 ? 0 : cap;
+        ctx = ctx < p.tok_base ? p.tok_base : cap;
     }
     return ctx;
+}
+
+// Partitions of this launch that sequence b's context needs.
+__device__ __forceinline__ int part_count(const DecodeParams& p, int ctx)
+{
+    return (ctx - p.tok_base + p.part_tokens - 1) / p.part_tokens;
+}
+
+// Workspace slot (row = b * H_q + h) of partition `part` of this launch.
+__device__ __forceinline__ size_t ws_slot(const DecodeParams& p, size_t row, int part)
+{
+    return row * p.slots + p.part_base + part;
 }
 
 // Byte address of 16-byte chunk `c` of row `t` in a tile stored as 128-byte-wide TMA

@@ -213,10 +213,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     const int hbase = g * p.G;
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
-    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
-    const int tok0 = part * p.part_tokens;
+    const int nparts = part_count(p, ctx);
+    const int tok0 = p.tok_base + part * p.part_tokens;
     if (tok0 >= ctx) {
-        if (part == 0) {
+        if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
             for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
         }
@@ -427,7 +427,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     // ---- epilogue: O^T row (D/8) r + 2 mt (+1 for the second half) -> [head][dim]
 #pragma unroll
     for (int hr = 0; hr < NHT; ++hr) l_run[hr] = warp_sum_quad(l_run[hr]);
-    const bool final_out = (nparts == 1);
+    const bool final_out = (p.part_base == 0 && nparts == 1);
     float* so = reinterpret_cast<float*>(smem);
     constexpr int SR = D + 4;
     __syncwarp();
@@ -456,7 +456,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     for (int i = lane; i < p.G * (D / 4); i += 32) {
         const int h = i / (D / 4), c4 = i % (D / 4);
         const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
-        const size_t off = final_out ? (row0 + h) * D : ((row0 + h) * p.max_parts + part) * D;
+        const size_t off = final_out ? (row0 + h) * D : ws_slot(p, row0 + h, part) * D;
         *reinterpret_cast<float4*>(dst + off + 4 * c4) = v;
     }
     if (!final_out && qd == 0) {
@@ -464,7 +464,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         for (int hr = 0; hr < NHT; ++hr) {
             const int h = r + 8 * hr;
             if (h < p.G)
-                *reinterpret_cast<float2*>(p.ws_ml + ((row0 + h) * p.max_parts + part) * 2) =
+                *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) =
                     make_float2(m_run[hr], l_run[hr]);
         }
     }

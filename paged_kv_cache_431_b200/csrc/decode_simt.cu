@@ -75,10 +75,10 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     const int hbase = g * G;
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
-    const int nparts = (ctx + p.part_tokens - 1) / p.part_tokens;
-    const int tok0 = part * p.part_tokens;
+    const int nparts = part_count(p, ctx);
+    const int tok0 = p.tok_base + part * p.part_tokens;
     if (tok0 >= ctx) {
-        if (part == 0) {
+        if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
             for (int i = lane; i < G * D; i += 32) o[i] = 0.f;
         }
@@ -271,7 +271,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     }
     __syncwarp();
     const size_t row0 = (size_t)b * p.H_q + hbase;
-    const bool final_out = nparts == 1;
+    const bool final_out = (p.part_base == 0 && nparts == 1);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const float inv = final_out ? 1.f / l_s[h] : 1.f;
@@ -279,11 +279,11 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         if (final_out) {
             *reinterpret_cast<float4*>(p.out + (row0 + h) * D + 4 * lane) = v;
         } else {
-            *reinterpret_cast<float4*>(p.ws_o + ((row0 + h) * p.max_parts + part) * D + 4 * lane) = v;
+            *reinterpret_cast<float4*>(p.ws_o + ws_slot(p, row0 + h, part) * D + 4 * lane) = v;
         }
     }
     if (!final_out && lane < G)
-        *reinterpret_cast<float2*>(p.ws_ml + ((row0 + lane) * p.max_parts + part) * 2) = make_float2(m_s[lane], l_s[lane]);
+        *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + lane, part) * 2) = make_float2(m_s[lane], l_s[lane]);
 }
 
 template <int G, bool BF16>

@@ -48,6 +48,8 @@ struct DecodeArgs {
     float* ws_ml;           // [B][H_q][max_parts][2]
     int32_t* status;
     int engine;             // 1 mma, 2 fma
+    int tok_base = 0;       // first token the partitions cover (cascade: the prefix length)
+    int part_base = 0;      // first workspace slot they write (cascade: 1)
 };
 
 int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
@@ -77,6 +79,13 @@ struct PrefillArgs {
     float scale;
     float* out;
     int32_t* status;
+    // tcgen05 form only: shared-prefix (cascade) pass of the decode.  With cascade_nkeys > 0
+    // the C positions are the decode batch, every row sees keys 0 .. cascade_nkeys-1, and the
+    // partial (o, m, l) goes to slot 0 of decode workspace rows of ws_slots slots.
+    int cascade_nkeys = 0;
+    int ws_slots = 0;
+    float* ws_o = nullptr;
+    float* ws_ml = nullptr;
 };
 
 int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);

@@ -49,6 +49,12 @@ struct TcParams {
     int32_t* status;
     int P0, C, H_q, H_kv, G, N;
     float scale_log2;
+    // Shared-prefix (cascade) form: the C "positions" are C sequences whose query rows all
+    // see the same nkeys keys (no causal mask); the unnormalized output and (m, l) go to
+    // slot 0 of the decode workspace rows [C][H_q][slots] instead of `out`.
+    int cascade, nkeys, slots;
+    float* ws_o;
+    float* ws_ml;
 };
 
 // ---- tcgen05 wrappers ------------------------------------------------------
@@ -186,8 +192,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
     const int pos_per_cta = kBM / p.G;
     const int i0 = blockIdx.x * pos_per_cta;                 // first chunk position of this CTA
     const int i_end = min(p.C, i0 + pos_per_cta);
-    const int seq_len = p.P0 + p.C;
-    const int kend = p.P0 + i_end;                           // exclusive key bound of the CTA's last row
+    const int seq_len = p.cascade ? p.nkeys : p.P0 + p.C;
+    const int kend = p.cascade ? p.nkeys : p.P0 + i_end;     // exclusive key bound of the CTA's last row
     const int ntiles = (kend + kBN - 1) / kBN;
     const int nblk_seq = (seq_len + kBlock - 1) / kBlock;
 
@@ -336,8 +342,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         const int hc = (warp - 2) >> 2;
         const int r = quarter * 32 + lane;                   // query row of this thread
         const int pos = i0 + r / p.G;
-        const int kmax = p.P0 + min(pos, p.C - 1) + 1;       // keys < kmax are visible
-        const int kmin_cta = p.P0 + i0 + 1;
+        const int kmax = p.cascade ? p.nkeys : p.P0 + min(pos, p.C - 1) + 1;   // keys < kmax are visible
+        const int kmin_cta = p.cascade ? p.nkeys : p.P0 + i0 + 1;
         const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t xcol = trow + 3 * kBN;                // exchange columns 384..387
         const uint32_t pair_bar = smem_u32(&bars.pair[quarter]);
@@ -380,21 +386,22 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
 
             const int key0 = t * kBN + (kBN / 2) * hc;
             const bool need_mask = t * kBN + kBN > kmin_cta;
-            float mx = -INFINITY;
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
             if (pos_scale) {        // max of the raw scores, scaled once
 #pragma unroll
                 for (int j = 0; j < kBN / 2; ++j) {
                     if (need_mask && key0 + j >= kmax) x[j] = -INFINITY;
-                    mx = fmaxf(mx, x[j]);
+                    m4[j & 3] = fmaxf(m4[j & 3], x[j]);
                 }
-                mx *= sl;
             } else {
 #pragma unroll
                 for (int j = 0; j < kBN / 2; ++j) {
                     x[j] = (need_mask && key0 + j >= kmax) ? -INFINITY : x[j] * sl;
-                    mx = fmaxf(mx, x[j]);
+                    m4[j & 3] = fmaxf(m4[j & 3], x[j]);
                 }
             }
+            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if (pos_scale) mx *= sl;
             mx = fmaxf(mx, exchange(mx, t));
             if (!ok) break;
             float m_new = m_used;
@@ -402,19 +409,22 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
 
             // P = 2^(score - m) as high + low 16-bit parts, computed before waiting for the
-            // previous P . V so the exponentials overlap the tensor cores.  bf16: the high
-            // part is the truncation (upper half of the fp32 word), the low part the exact
-            // remainder rounded to bf16.
+            // previous P . V so the exponentials overlap the tensor cores.  bf16: the high part
+            // is the truncation (upper half of the fp32 word), the low part the truncated
+            // remainder; both are byte permutes, so no conversion instruction is issued.
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             float sum = 0.f;
             uint32_t ph[kBN / 4], pl[kBN / 4];
 #pragma unroll
             for (int e = 0; e < kBN / 4; ++e) {
-                const float p0 = ex2(fmaf(x[2 * e], slx, -mref)), p1 = ex2(fmaf(x[2 * e + 1], slx, -mref));
+                const float a0 = fmaf(x[2 * e], slx, -mref), a1 = fmaf(x[2 * e + 1], slx, -mref);
+                const float p0 = ex2(a0), p1 = ex2(a1);
                 if constexpr (BF16) {
                     const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
                     ph[e] = __byte_perm(u0, u1, 0x7632);
-                    pl[e] = pack2<true>(p0 - __uint_as_float(u0 & 0xffff0000u), p1 - __uint_as_float(u1 & 0xffff0000u));
+                    const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                    pl[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
                 } else {
                     ph[e] = pack2<false>(p0, p1);
                     const float2 back = unpack2<false>(ph[e]);
@@ -480,8 +490,11 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (ntiles - 1) & 1, &s_abort, p.status))) {
             tc_fence_after();
             const bool valid = pos < p.C;
-            const float inv = 1.f / l_tot;
-            float* orow = p.out + ((size_t)pos * p.H_q + g * p.G + (r % p.G)) * kD + (kD / 2) * hc;
+            const float inv = p.cascade ? 1.f : 1.f / l_tot;
+            const size_t qrow = (size_t)pos * p.H_q + g * p.G + (r % p.G);
+            float* orow = (p.cascade ? p.ws_o + qrow * p.slots * kD : p.out + qrow * kD) + (kD / 2) * hc;
+            if (p.cascade && valid && hc == 0)
+                *reinterpret_cast<float2*>(p.ws_ml + qrow * p.slots * 2) = make_float2(m_used, l_tot);
 #pragma unroll 1
             for (int c = 0; c < kD / 64; ++c) {
                 float o[32];
@@ -538,6 +551,11 @@ int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtens
     p.G = a.G;
     p.N = a.N;
     p.scale_log2 = a.scale * kLog2e;
+    p.cascade = a.cascade_nkeys > 0;
+    p.nkeys = a.cascade_nkeys;
+    p.slots = a.ws_slots;
+    p.ws_o = a.ws_o;
+    p.ws_ml = a.ws_ml;
     auto kern = a.kv_dtype == PKV_BF16 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
         return PKV_ERR_CUDA;

@@ -17,7 +17,7 @@ from . import build as _build
 BLOCK_SIZE = 16
 F16, BF16, INT8, INT4, FP8E4M3 = 0, 1, 2, 3, 4
 QUANTIZED = (INT8, INT4, FP8E4M3)
-DEV_BAD_BLOCK, DEV_BAD_SLOT, DEV_BAD_LENGTH, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEV_BAD_BLOCK, DEV_BAD_SLOT, DEV_BAD_LENGTH, DEV_TIMEOUT, DEV_BAD_PREFIX = 0x1, 0x2, 0x4, 0x8, 0x10
 ENGINE_AUTO, ENGINE_MMA, ENGINE_FMA2, ENGINE_FMA = 0, 1, 2, 3
 
 _TORCH16 = {F16: torch.float16, BF16: torch.bfloat16}
@@ -239,6 +239,43 @@ def paged_decode_attn(pool: KVPool, layer: int, q: torch.Tensor, block_tables: t
                                    block_tables.shape[1], _ptr(context_lens), B, H_q, max_context_len,
                                    float(scale), _ptr(out), _ptr(workspace), ws_bytes,
                                    _opts(engine, partition_tokens), _stream(stream)), "paged_decode_attn")
+    return out
+
+
+def paged_decode_cascade_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int, max_context_len: int,
+                                        shared_prefix_len: int, engine: int = 0, partition_tokens: int = 0) -> int:
+    L = lib()
+    fn = L.paged_decode_cascade_workspace_bytes
+    fn.restype = ctypes.c_size_t
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    return int(fn(pool.handle, num_seqs, num_q_heads, max_context_len, shared_prefix_len,
+                  _opts(engine, partition_tokens)))
+
+
+def paged_decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, block_tables: torch.Tensor,
+                              context_lens: torch.Tensor, scale: float, max_context_len: int,
+                              shared_prefix_len: int, out: torch.Tensor | None = None,
+                              workspace: torch.Tensor | None = None, engine: int = 0, partition_tokens: int = 0,
+                              stream=None) -> torch.Tensor:
+    """Decode attention for a batch whose tables all start with the same shared_prefix_len
+    tokens (row 0's blocks): the prefix is attended once per KV group on the tensor cores."""
+    L = lib()
+    fn = L.paged_decode_attn_cascade
+    P, i32 = ctypes.c_void_p, ctypes.c_int
+    fn.restype = i32
+    fn.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, i32, ctypes.c_float, P, P, ctypes.c_size_t, P, P]
+    B, H_q, d = q.shape
+    if out is None:
+        out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
+    need = paged_decode_cascade_workspace_bytes(pool, B, H_q, max_context_len, shared_prefix_len, engine,
+                                                partition_tokens)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_tables), block_tables.shape[1],
+              _ptr(context_lens), B, H_q, max_context_len, shared_prefix_len, float(scale), _ptr(out),
+              _ptr(workspace), ws_bytes, _opts(engine, partition_tokens), _stream(stream)),
+           "paged_decode_attn_cascade")
     return out
 
 

@@ -41,7 +41,9 @@ MUTANTS = [
     ("table_index", "int blk = table[t / ORC_BLOCK], off = t % ORC_BLOCK;\n        if (blk < 0",
      "int blk = table[t % ORC_BLOCK < 0 ? 0 : t / ORC_BLOCK / 2], off = t % ORC_BLOCK;\n        if (blk < 0",
      lambda: pins.test_block_table_figure(_golden())),
-    ("causal_off_by_one", "ctx_before + i + 1, (double)scale", "ctx_before + i, (double)scale",
+    ("window_off_by_one", "? n - window : 0;", "? n - window + 1 : 0;",
+     lambda: pins.test_sliding_window_equals_library_attention_over_the_last_positions(5)),
+    ("causal_off_by_one", "window), ctx_before + i + 1,", "window), ctx_before + i,",
      lambda: pins.test_prefill_chunk_rows_equal_decode_and_causal_library()),
     ("size_factor_two", "return (int64_t)2 * layers", "return (int64_t)layers",
      lambda: pins.test_bytes_per_token_worked_values(_golden())),

@@ -300,6 +300,62 @@ def test_prefill_chunk_rows_equal_decode_and_causal_library():
             assert np.allclose(out[i, h], ref, rtol=1e-11, atol=1e-12)
 
 
+# ------------------------------------------------------------ sliding window --
+
+@pytest.mark.parametrize("window", [1, 5, 16, 17, 40])
+def test_sliding_window_equals_library_attention_over_the_last_positions(window):
+    """A window of w ("The KV cache" on the continuous-batching page: sliding-window
+    attention layers) sees positions n-w .. n-1 of a decode of length n and
+    p-w+1 .. p for chunk row at position p: library softmax attention over exactly those
+    rows of the logical sequence.  w = 1 returns the last V row exactly."""
+    rng = np.random.default_rng(100 + window)
+    H_kv, G, d = 2, 2, 16
+    H_q = H_kv * G
+    lens = [0, 1, 3, 16, 17, 33, 64]
+    W = max(oracle.blocks_for_tokens(n) for n in lens)
+    N = sum(oracle.blocks_for_tokens(n) for n in lens) + 3
+    perm = rng.permutation(N)
+    tables, cur, Ks, Vs = np.full((len(lens), W), -1, np.int32), 0, [], []
+    for b, n in enumerate(lens):
+        nb = oracle.blocks_for_tokens(n)
+        tables[b, :nb] = perm[cur:cur + nb]
+        cur += nb
+        K, V = random_logical(rng, n, H_kv, d)
+        Ks.append(K)
+        Vs.append(V)
+    pool = build_pool_from_logical(Ks, Vs, tables, N, H_kv, d)
+    q = rng.standard_normal((len(lens), H_q, d)).astype(np.float16)
+    out = oracle.paged_decode(pool, f16_bits(q), oracle.F16, tables, lens, 0.25, window=window)
+    for b, n in enumerate(lens):
+        lo = max(0, n - window)
+        for h in range(H_q):
+            if n == 0:
+                assert not out[b, h].any()
+                continue
+            ref = library_attention(q[b, h].astype(np.float64), Ks[b][lo:, h // G].astype(np.float64),
+                                    Vs[b][lo:, h // G].astype(np.float64), 0.25)
+            assert np.allclose(out[b, h], ref, rtol=1e-11, atol=1e-12), (b, h)
+            if window == 1:
+                assert np.array_equal(out[b, h], Vs[b][n - 1, h // G].astype(np.float64))
+    # a window at least as long as every context is no window at all
+    full = oracle.paged_decode(pool, f16_bits(q), oracle.F16, tables, lens, 0.25)
+    wide = oracle.paged_decode(pool, f16_bits(q), oracle.F16, tables, lens, 0.25, window=64)
+    assert np.array_equal(full, wide)
+    # chunk rows: row i at position P0 + i sees max(0, P0 + i + 1 - w) .. P0 + i
+    P0, C = 20, 13
+    K, V = random_logical(rng, P0 + C, H_kv, d)
+    table = [4, 0, 2]
+    cpool = build_pool_from_logical([K], [V], [table], 6, H_kv, d)
+    qc = rng.standard_normal((C, H_q, d)).astype(np.float16)
+    cout = oracle.paged_prefill_chunk(cpool, f16_bits(qc), oracle.F16, table, P0, 0.25, window=window)
+    for i in range(C):
+        lo = max(0, P0 + i + 1 - window)
+        for h in range(H_q):
+            ref = library_attention(qc[i, h].astype(np.float64), K[lo:P0 + i + 1, h // G].astype(np.float64),
+                                    V[lo:P0 + i + 1, h // G].astype(np.float64), 0.25)
+            assert np.allclose(cout[i, h], ref, rtol=1e-11, atol=1e-12)
+
+
 # ------------------------------------------------------------------ 16-bit append --
 
 def test_append_16bit_is_a_slot_copy():
