@@ -153,10 +153,16 @@ typedef struct {
                                   PKV_ERR_UNSUPPORTED); kept to measure the FP32-pipe form of the decode */
     int32_t partition_tokens;  /* tokens per split-K partition; 0 = chosen from the workload; else a
                                   multiple of 16 in [64, 16384] */
+    int32_t sliding_window;    /* 0 = attend to the whole context; w > 0 = sliding-window attention
+                                  ([KVB] "The KV cache": sliding-window or local attention layers):
+                                  the query (position context_len - 1) sees only positions
+                                  context_len - w .. context_len - 1; blocks wholly before the window
+                                  are not read.  Not with paged_decode_attn_cascade. */
 } pkv_decode_opts;
 
 /* Workspace paged_decode_attn needs for these sizes and options (bytes): per (sequence,
- * query head, partition) a head_dim + 2 fp32 partial (o, m, l). */
+ * query head, partition) a head_dim + 2 fp32 partial (o, m, l).  With a sliding window the
+ * partitions cover at most window + 15 tokens per sequence. */
 PKV_API size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads,
                                     int max_context_len, const pkv_decode_opts* opts);
 
@@ -164,7 +170,8 @@ PKV_API size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int n
  * paged_decode_attn -- one new query token per sequence attends to all its cached tokens,
  * following its block table ([KVB] "Paged attention": the attention kernel follows the
  * block table; [KVG] "What it is": the cache holds K/V of every previous token).
- *   out[b][h][:] = sum_t softmax_t(scale * q[b][h] . K_b[t][h/G]) V_b[t][h/G],  t < context_lens[b]
+ *   out[b][h][:] = sum_t softmax_t(scale * q[b][h] . K_b[t][h/G]) V_b[t][h/G],  lo_b <= t < context_lens[b]
+ * (lo_b = 0, or max(0, context_lens[b] - w) with opts->sliding_window = w)
  * with K_b[t] = pool tile (block_tables[b][t/16], kv head) row t%16, dequantized as
  * code * scale for quantized pools.  A context length of 0 gives a zero row.
  *   q [device]: [num_seqs][num_q_heads][head_dim], q_dtype PKV_F16 or PKV_BF16 (for 16-bit
@@ -175,7 +182,8 @@ PKV_API size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int n
  *   max_context_len [host]: sizes the split-K grid.
  *   out [device]: fp32 [num_seqs][num_q_heads][head_dim].
  *   workspace [device]: paged_decode_workspace_bytes(...) bytes, 16-byte aligned.
- * num_q_heads / num_kv_heads must be an integer G in [1, 16].
+ * num_q_heads / num_kv_heads must be an integer G >= 1 (MHA G = 1 .. MQA H_kv = 1; groups
+ * of more than 16 query heads are split over several CTAs that read the same K/V tiles).
  */
 PKV_API int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype,
                       const int32_t* block_tables, int block_table_width,
@@ -263,6 +271,19 @@ PKV_API int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, 
                              const int32_t* block_table, int block_table_width,
                              int ctx_before, int chunk_len, int num_q_heads, float scale,
                              float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * paged_prefill_chunk_attn_window -- paged_prefill_chunk_attn with sliding-window
+ * attention ([KVB] "The KV cache": sliding-window or local attention layers): query row i
+ * (position ctx_before + i) sees only positions max(0, ctx_before + i + 1 - sliding_window)
+ * .. ctx_before + i; key tiles wholly before a CTA's windows are not read.
+ * sliding_window 0 is paged_prefill_chunk_attn.  No workspace.  Rows with a window run on
+ * the warp-level mma.sync form of the kernel.
+ */
+PKV_API int paged_prefill_chunk_attn_window(pkv_pool_t pool, int layer, const void* q, int q_dtype,
+                                            const int32_t* block_table, int block_table_width,
+                                            int ctx_before, int chunk_len, int num_q_heads, float scale,
+                                            int sliding_window, float* out, void* stream);
 
 /*
  * kv_copy_blocks -- copy-on-write at divergence ([KVB] "Paged attention": blocks shared

@@ -231,9 +231,13 @@ int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, int src_
 static int decode_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, const pkv_decode_opts* opts, int* P,
                                int* max_parts)
 {
-    *P = choose_partition(num_seqs, pool->d.num_kv_heads, max_ctx, pool->row_bytes, opts);
+    const int window = opts ? opts->sliding_window : 0;
+    if (window < 0) return PKV_ERR_ARG;
+    // with a window a sequence's partitions start at the block holding ctx - window
+    const int span = (window > 0 && max_ctx > window + PKV_BLOCK_SIZE - 1) ? window + PKV_BLOCK_SIZE - 1 : max_ctx;
+    *P = choose_partition(num_seqs, pool->d.num_kv_heads, span, pool->row_bytes, opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
-    *max_parts = max_ctx > 0 ? (max_ctx + *P - 1) / *P : 1;
+    *max_parts = span > 0 ? (span + *P - 1) / *P : 1;
     return PKV_OK;
 }
 
@@ -259,7 +263,7 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
         return PKV_ERR_ARG;
     if (num_q_heads % d.num_kv_heads) return PKV_ERR_SHAPE;
     const int G = num_q_heads / d.num_kv_heads;
-    if (G > 16) return PKV_ERR_UNSUPPORTED;
+    if ((long long)d.num_kv_heads * ((G + 15) / 16) > 65535) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
     if (!q || !block_tables || !context_lens || !out) return PKV_ERR_NULL;
     if (q_dtype != PKV_F16 && q_dtype != PKV_BF16) return PKV_ERR_DTYPE;
@@ -302,6 +306,7 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     a.ws_ml = need ? ws + (size_t)num_seqs * num_q_heads * parts * d.head_dim : nullptr;
     a.status = d.device_status;
     a.engine = engine;
+    a.window = opts ? opts->sliding_window : 0;
     return launch_decode(a, tmk, tmv, static_cast<cudaStream_t>(stream));
 }
 
@@ -356,6 +361,7 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
         (long long)block_table_width * PKV_BLOCK_SIZE < shared_prefix_len)
         return PKV_ERR_SHAPE;
     if (!cascade_shape_ok(pool, num_q_heads, max_context_len, shared_prefix_len)) return PKV_ERR_UNSUPPORTED;
+    if (opts && opts->sliding_window != 0) return PKV_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PKV_OK;
     if (!q || !block_tables || !context_lens || !out) return PKV_ERR_NULL;
     if (q_dtype != d.kv_dtype) return PKV_ERR_DTYPE;
@@ -449,7 +455,16 @@ int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, int q_dt
 {
     (void)workspace;
     (void)workspace_bytes;
+    return paged_prefill_chunk_attn_window(pool, layer, q, q_dtype, block_table, block_table_width, ctx_before,
+                                           chunk_len, num_q_heads, scale, 0, out, stream);
+}
+
+int paged_prefill_chunk_attn_window(pkv_pool_t pool, int layer, const void* q, int q_dtype,
+                                    const int32_t* block_table, int block_table_width, int ctx_before, int chunk_len,
+                                    int num_q_heads, float scale, int sliding_window, float* out, void* stream)
+{
     if (!pool) return PKV_ERR_NULL;
+    if (sliding_window < 0) return PKV_ERR_ARG;
     const pkv_pool_desc& d = pool->d;
     if (layer < 0 || layer >= d.num_layers || ctx_before < 0 || chunk_len < 0 || num_q_heads <= 0 ||
         block_table_width <= 0)
@@ -480,7 +495,8 @@ int paged_prefill_chunk_attn(pkv_pool_t pool, int layer, const void* q, int q_dt
     a.scale = scale;
     a.out = out;
     a.status = d.device_status;
-    if (prefill_tc_supported(a.d, a.G, a.kv_dtype)) {
+    a.window = sliding_window;
+    if (sliding_window == 0 && prefill_tc_supported(a.d, a.G, a.kv_dtype)) {
         CUtensorMap tmq;
         auto enc = tensor_map_encoder();
         if (!enc || !make_q_map(&tmq, q, chunk_len, num_q_heads, a.G, enc)) return PKV_ERR_CUDA;

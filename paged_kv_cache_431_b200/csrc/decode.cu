@@ -54,17 +54,20 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 
     pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
     const int lane = threadIdx.x;
-    const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int part = blockIdx.x, b = blockIdx.z;
+    const int g = blockIdx.y / p.hgroups, hg = blockIdx.y - g * p.hgroups;   // KV head, group of 16 heads
+    const int GC = min(16, p.G - 16 * hg);                                   // query heads of this CTA
     const int r = lane >> 2, qd = lane & 3;
-    const int hbase = g * p.G;
+    const int hbase = g * p.G + 16 * hg;
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
     const int nparts = part_count(p, ctx);
-    const int tok0 = p.tok_base + part * p.part_tokens;
+    const int tok0 = seq_base(p, ctx) + part * p.part_tokens;
+    const int lo = visible_lo(p, ctx);   // tokens before lo are outside the window
     if (tok0 >= ctx) {
         if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
-            for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
+            for (int i = lane; i < GC * D; i += 32) o[i] = 0.f;
         }
         return;
     }
@@ -109,7 +112,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     {
         const uint32_t* q32 = reinterpret_cast<const uint32_t*>(
             static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D);
-        const bool r0 = r < p.G, r1 = (NHT == 2) && (r + 8 < p.G);
+        const bool r0 = r < GC, r1 = (NHT == 2) && (r + 8 < GC);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             qa[ks][0] = r0 ? __ldg(q32 + (r * D + 16 * ks + 2 * qd) / 2) : 0u;
@@ -140,6 +143,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
         const uint32_t vb = kb + Cfg::TILE;
         const int nv = min(kBlock, ntok - j * kBlock);
+        const int nlo = lo - (tok0 + j * kBlock);   // tokens of this tile before the window: < nlo
 
         // S = Q . K^T  (two n-tiles of 8 tokens)
         float sc[2][4];
@@ -170,7 +174,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tok = nt * 8 + 2 * qd + e;
-                    x[nt][e] = tok < nv ? sc[nt][2 * hr + e] * sl : -INFINITY;
+                    x[nt][e] = (tok < nv && tok >= nlo) ? sc[nt][2 * hr + e] * sl : -INFINITY;
                     mx = fmaxf(mx, x[nt][e]);
                 }
             mx = warp_max_quad(mx);
@@ -218,9 +222,10 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
             }
 
         uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
-        if (nv < kBlock) {   // zero V of past-the-end tokens (their P is 0, their V may be stale)
-            keep01 = (2 * qd < nv ? 0x0000ffffu : 0u) | (2 * qd + 1 < nv ? 0xffff0000u : 0u);
-            keep23 = (8 + 2 * qd < nv ? 0x0000ffffu : 0u) | (9 + 2 * qd < nv ? 0xffff0000u : 0u);
+        if (nv < kBlock || nlo > 0) {   // zero V outside [nlo, nv): P is 0 there, V may be stale
+            auto in = [&](int t) { return t >= nlo && t < nv; };
+            keep01 = (in(2 * qd) ? 0x0000ffffu : 0u) | (in(2 * qd + 1) ? 0xffff0000u : 0u);
+            keep23 = (in(8 + 2 * qd) ? 0x0000ffffu : 0u) | (in(9 + 2 * qd) ? 0xffff0000u : 0u);
         }
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
@@ -279,13 +284,13 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     __syncwarp();
     const size_t row0 = (size_t)b * p.H_q + hbase;
     if (final_out) {
-        for (int i = lane; i < p.G * (D / 4); i += 32) {
+        for (int i = lane; i < GC * (D / 4); i += 32) {
             const int h = i / (D / 4), c4 = i % (D / 4);
             const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
             *reinterpret_cast<float4*>(p.out + (row0 + h) * D + 4 * c4) = v;
         }
     } else {
-        for (int i = lane; i < p.G * (D / 4); i += 32) {
+        for (int i = lane; i < GC * (D / 4); i += 32) {
             const int h = i / (D / 4), c4 = i % (D / 4);
             const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
             *reinterpret_cast<float4*>(p.ws_o + ws_slot(p, row0 + h, part) * D + 4 * c4) = v;
@@ -294,7 +299,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll
             for (int hr = 0; hr < NHT; ++hr) {
                 const int h = r + 8 * hr;
-                if (h < p.G) {
+                if (h < GC) {
                     float2 ml = make_float2(m_run[hr], l_run[hr]);
                     *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) = ml;
                 }
@@ -409,11 +414,13 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.part_base = a.part_base;
     p.slots = a.part_base + a.max_parts;
     p.prefix_blocks = a.part_base ? a.tok_base / kBlock : 0;
+    p.window = a.window;
+    p.hgroups = (a.G + 15) / 16;
     p.q_bf16 = a.q_dtype == PKV_BF16;
     p.scale_log2 = a.scale * kLog2e;
 
-    const dim3 grid(a.max_parts, a.H_kv, a.B);
-    const int nht = a.G <= 8 ? 1 : 2;
+    const dim3 grid(a.max_parts, a.H_kv * p.hgroups, a.B);
+    const int nht = a.G <= 8 ? 1 : 2;   // 8 or 16 query heads per CTA
     int rc = PKV_ERR_UNSUPPORTED;
     if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && (a.engine == 2 || a.engine == 3)) {
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))

@@ -25,15 +25,18 @@ struct DecodeParams {
     // tok_base = prefix length, part_base = 1 (slot 0 holds the prefix's partial).
     int tok_base, part_base, slots;
     int prefix_blocks;      // cascade: table entries every sequence must share with row 0
+    int window;             // sliding window: tokens a query sees (0: the whole context)
+    int hgroups;            // CTAs per KV head, 16 query heads each (G > 16 takes several)
     int q_bf16;             // q dtype: 1 bf16, 0 f16
     float scale_log2;
 };
 
-// Context length of sequence b, clamped to what the table and the grid can cover.
+// Context length of sequence b, clamped to what the table and the grid can cover (with a
+// window the grid covers any context: a query reads at most window + 15 tokens' blocks).
 __device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool report)
 {
     int ctx = p.ctx_lens[b];
-    const int cap = min(p.W * kBlock, p.tok_base + p.max_parts * p.part_tokens);
+    const int cap = p.window ? p.W * kBlock : min(p.W * kBlock, p.tok_base + p.max_parts * p.part_tokens);
     if (ctx < p.tok_base || ctx > cap) {
         if (report) flag_status(p.status, PKV_DEV_BAD_LENGTH);
         ctx = ctx < p.tok_base ? p.tok_base : cap;
@@ -41,10 +44,22 @@ __device__ __forceinline__ int checked_ctx(const DecodeParams& p, int b, bool re
     return ctx;
 }
 
+// First token the query sees: ctx - window with a sliding window, else 0.
+__device__ __forceinline__ int visible_lo(const DecodeParams& p, int ctx)
+{
+    return (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
+}
+
+// First token of partition 0: the prefix end (cascade), or the block holding visible_lo.
+__device__ __forceinline__ int seq_base(const DecodeParams& p, int ctx)
+{
+    return p.window > 0 ? (visible_lo(p, ctx) & ~(kBlock - 1)) : p.tok_base;
+}
+
 // Partitions of this launch that sequence b's context needs.
 __device__ __forceinline__ int part_count(const DecodeParams& p, int ctx)
 {
-    return (ctx - p.tok_base + p.part_tokens - 1) / p.part_tokens;
+    return (ctx - seq_base(p, ctx) + p.part_tokens - 1) / p.part_tokens;
 }
 
 // Workspace slot (row = b * H_q + h) of partition `part` of this launch.

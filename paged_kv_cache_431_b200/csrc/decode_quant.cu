@@ -208,17 +208,20 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 
     pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
     const int lane = threadIdx.x;
-    const int part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int part = blockIdx.x, b = blockIdx.z;
+    const int g = blockIdx.y / p.hgroups, hg = blockIdx.y - g * p.hgroups;   // KV head, group of 16 heads
+    const int GC = min(16, p.G - 16 * hg);                                   // query heads of this CTA
     const int r = lane >> 2, qd = lane & 3;
-    const int hbase = g * p.G;
+    const int hbase = g * p.G + 16 * hg;
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
     const int nparts = part_count(p, ctx);
-    const int tok0 = p.tok_base + part * p.part_tokens;
+    const int tok0 = seq_base(p, ctx) + part * p.part_tokens;
+    const int lo = visible_lo(p, ctx);   // tokens before lo are outside the window
     if (tok0 >= ctx) {
         if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
-            for (int i = lane; i < p.G * D; i += 32) o[i] = 0.f;
+            for (int i = lane; i < GC * D; i += 32) o[i] = 0.f;
         }
         return;
     }
@@ -271,7 +274,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             const uint16_t u = __ldg(qh + row * D + dim);
             return bf ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
         };
-        const bool r0 = r < p.G, r1 = (NHT == 2) && (r + 8 < p.G);
+        const bool r0 = r < GC, r1 = (NHT == 2) && (r + 8 < GC);
 #pragma unroll
         for (int ks = 0; ks < Cfg::KS; ++ks) {
             const int d0 = kdim<DT, D>(ks, qd, 0), d1 = kdim<DT, D>(ks, qd, 1);
@@ -303,6 +306,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
         const uint32_t vb = kb + Cfg::TILE;
         const int nv = min(kBlock, ntok - j * kBlock);
+        const int nlo = lo - (tok0 + j * kBlock);   // tokens of this tile before the window: < nlo
         const float2 sc_kv = tsc[j];
 
         // S = Q . K^T, token 8 nt + r of the tile in n-tile nt
@@ -333,7 +337,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tok = nt * 8 + 2 * qd + e;
-                    x[nt][e] = tok < nv ? sc[nt][2 * hr + e] * sl : -INFINITY;
+                    x[nt][e] = (tok < nv && tok >= nlo) ? sc[nt][2 * hr + e] * sl : -INFINITY;
                     mx = fmaxf(mx, x[nt][e]);
                 }
             mx = warp_max_quad(mx);
@@ -379,9 +383,11 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             }
 
         uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
-        if (nv < kBlock) {
-            keep01 = (2 * qd < nv ? 0x0000ffffu : 0u) | (2 * qd + 1 < nv ? 0xffff0000u : 0u);
-            keep23 = (8 + 2 * qd < nv ? 0x0000ffffu : 0u) | (9 + 2 * qd < nv ? 0xffff0000u : 0u);
+        const bool partial = nv < kBlock || nlo > 0;
+        if (partial) {   // zero V outside [nlo, nv): P is 0 there, V may be stale
+            auto in = [&](int t) { return t >= nlo && t < nv; };
+            keep01 = (in(2 * qd) ? 0x0000ffffu : 0u) | (in(2 * qd + 1) ? 0xffff0000u : 0u);
+            keep23 = (in(8 + 2 * qd) ? 0x0000ffffu : 0u) | (in(9 + 2 * qd) ? 0xffff0000u : 0u);
         }
         uint32_t wa[Cfg::VRUN / 4], wb[Cfg::VRUN / 4], wc[Cfg::VRUN / 4], wd[Cfg::VRUN / 4];
         load_run<ROW, SWZ, Cfg::VRUN>(wa, vb, 2 * qd, r * Cfg::VRUN);
@@ -396,7 +402,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 #pragma unroll
             for (int jj = 0; jj < MT_PER_WORD; ++jj) {
                 const int mt = k * MT_PER_WORD + jj;
-                if (nv < kBlock) {   // zero V of past-the-end tokens
+                if (partial) {   // zero V outside the visible tokens
                     va[jj][0] &= keep01;
                     va[jj][1] &= keep01;
                     va[jj][2] &= keep23;
@@ -453,7 +459,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     __syncwarp();
     const size_t row0 = (size_t)b * p.H_q + hbase;
     float* dst = final_out ? p.out : p.ws_o;
-    for (int i = lane; i < p.G * (D / 4); i += 32) {
+    for (int i = lane; i < GC * (D / 4); i += 32) {
         const int h = i / (D / 4), c4 = i % (D / 4);
         const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
         const size_t off = final_out ? (row0 + h) * D : ws_slot(p, row0 + h, part) * D;
@@ -463,7 +469,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 #pragma unroll
         for (int hr = 0; hr < NHT; ++hr) {
             const int h = r + 8 * hr;
-            if (h < p.G)
+            if (h < GC)
                 *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) =
                     make_float2(m_run[hr], l_run[hr]);
         }

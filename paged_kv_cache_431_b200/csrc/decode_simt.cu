@@ -76,7 +76,8 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
 
     const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
     const int nparts = part_count(p, ctx);
-    const int tok0 = p.tok_base + part * p.part_tokens;
+    const int tok0 = seq_base(p, ctx) + part * p.part_tokens;
+    const int lo = visible_lo(p, ctx);   // tokens before lo are outside the window
     if (tok0 >= ctx) {
         if (part == 0 && p.part_base == 0) {   // empty context: a zero row
             float* o = p.out + ((size_t)b * p.H_q + hbase) * D;
@@ -148,6 +149,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
         const uint32_t vb = kb + Cfg::TILE;
         const int nv = min(kBlock, ntok - j * kBlock);
+        const int nlo = lo - (tok0 + j * kBlock);   // tokens of this tile before the window: < nlo
 
         // partial scores: this lane's 8 dims, 8 tokens, G heads
         float acc[G * 8];
@@ -197,7 +199,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         float mx = -INFINITY;
 #pragma unroll
         for (int f = 0; f < NF; ++f) {
-            x[f] = t0 + f < nv ? acc[f] * sl : -INFINITY;
+            x[f] = (t0 + f < nv && t0 + f >= nlo) ? acc[f] * sl : -INFINITY;
             mx = fmaxf(mx, x[f]);
         }
 #pragma unroll
@@ -226,7 +228,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             for (int k = 0; k < 4; ++k) o[h][k] *= a;
         }
         const uint32_t vaddr_off = (uint32_t)((lane & 1) * 8);
-        for (int t = 0; t < nv; ++t) {
+        for (int t = max(nlo, 0); t < nv; ++t) {
             uint32_t w0, w1;
             asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(swz128(vb, t, lane >> 1) + vaddr_off));
             const float2 v01 = unpack2<BF16>(w0), v23 = unpack2<BF16>(w1);

@@ -50,6 +50,7 @@ struct DecodeArgs {
     int engine;             // 1 mma, 2 fma
     int tok_base = 0;       // first token the partitions cover (cascade: the prefix length)
     int part_base = 0;      // first workspace slot they write (cascade: 1)
+    int window = 0;         // sliding window (tokens a query sees), 0 = whole context
 };
 
 int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
@@ -82,6 +83,7 @@ struct PrefillArgs {
     // tcgen05 form only: shared-prefix (cascade) pass of the decode.  With cascade_nkeys > 0
     // the C positions are the decode batch, every row sees keys 0 .. cascade_nkeys-1, and the
     // partial (o, m, l) goes to slot 0 of decode workspace rows of ws_slots slots.
+    int window = 0;         // sliding window (warp-level form only)
     int cascade_nkeys = 0;
     int ws_slots = 0;
     float* ws_o = nullptr;

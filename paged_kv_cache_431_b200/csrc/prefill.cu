@@ -41,6 +41,7 @@ struct PrefillParams {
     float* out;
     int32_t* status;
     int W, P0, C, H_q, H_kv, G, N;
+    int window;             // sliding window (keys a row sees, itself included); 0 = all earlier
     float scale_log2;
 };
 
@@ -69,6 +70,9 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const int i_last = min(p.C - 1, (row_cta + kRows - 1) / p.G);
     const int kend_cta = p.P0 + i_last + 1;
     const int ntiles = (kend_cta + kKeys - 1) / kKeys;
+    // with a sliding window, tiles wholly before the first row's window are skipped
+    const int lo_cta = p.window > 0 ? max(0, p.P0 + min(p.C - 1, row_cta / p.G) + 1 - p.window) : 0;
+    const int t_begin = lo_cta / kKeys;
     const int seq_len = p.P0 + p.C;
     const int nblk_seq = (seq_len + kBlock - 1) / kBlock;
 
@@ -82,8 +86,8 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     }
     __syncthreads();
 
-    auto issue = [&](int t) {
-        const int s = t % Cfg::STAGES;
+    auto issue = [&](int t) {   // t: key tile; its ring stage counts from t_begin
+        const int s = (t - t_begin) % Cfg::STAGES;
         const uint32_t bar = smem_u32(&bars[s]);
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
@@ -92,9 +96,10 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
             const int lb = t * 4 + kb;        // logical block of the sequence
-            // past the sequence's last block: load block 0 (in bounds); those keys are
-            // masked and their V zeroed below
-            int blk = lb < nblk_seq ? p.table[lb] : 0;
+            // past the sequence's last block, or wholly before every row's window (an engine
+            // may have released it): load block 0 (in bounds); those keys are masked and
+            // their V zeroed below
+            int blk = (lb < nblk_seq && (lb + 1) * kBlock > lo_cta) ? p.table[lb] : 0;
             if ((unsigned)blk >= (unsigned)p.N) {
                 flag_status(p.status, PKV_DEV_BAD_BLOCK);
                 blk = 0;
@@ -111,7 +116,7 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         }
     };
     if (tid == 0) {
-        for (int t = 0; t < min(Cfg::STAGES, ntiles); ++t) issue(t);
+        for (int t = t_begin; t < min(t_begin + Cfg::STAGES, ntiles); ++t) issue(t);
     }
 
     // this warp's rows: r0 = row of lane group rg, r1 = r0 + 8
@@ -119,6 +124,8 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const bool v0 = r0 < rows_total, v1 = r1 < rows_total;
     const int i0 = v0 ? r0 / p.G : 0, i1 = v1 ? r1 / p.G : 0;
     const int kmax0 = p.P0 + i0 + 1, kmax1 = p.P0 + i1 + 1;   // exclusive key bounds
+    const int klo0 = p.window > 0 ? max(0, kmax0 - p.window) : 0;   // first visible keys
+    const int klo1 = p.window > 0 ? max(0, kmax1 - p.window) : 0;
     uint32_t qa[D / 16][4];
     {
         const uint16_t* qb = static_cast<const uint16_t*>(p.q);
@@ -142,15 +149,20 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const float sl = p.scale_log2;
     // the warp's smallest key bound: tiles entirely below it need no causal mask
     const int kmin_warp = p.P0 + min(p.C - 1, (row_cta + warp * 16) / p.G) + 1;
+    // the warp's window starts: tiles wholly at or above the largest need no window mask,
+    // tiles wholly below the smallest are skipped
+    const int kwin_lo = p.window > 0 ? max(0, kmin_warp - p.window) : 0;
+    const int kwin_hi = p.window > 0 ? max(0, p.P0 + min(p.C - 1, (row_cta + warp * 16 + 15) / p.G) + 1 - p.window) : 0;
 
-    for (int t = 0; t < ntiles; ++t) {
-        const int s = t % Cfg::STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (t / Cfg::STAGES) & 1)) atomicExch(&s_fail, 1);
+    for (int t = t_begin; t < ntiles; ++t) {
+        const int s = (t - t_begin) % Cfg::STAGES;
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), ((t - t_begin) / Cfg::STAGES) & 1)) atomicExch(&s_fail, 1);
         const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
         const uint32_t vb = kb + Cfg::KBYTES;
         const int key0 = t * kKeys;
 
-        if (key0 < p.P0 + min(p.C - 1, (row_cta + warp * 16 + 15) / p.G) + 1) {   // warp has work here
+        if (key0 < p.P0 + min(p.C - 1, (row_cta + warp * 16 + 15) / p.G) + 1 &&
+            key0 + kKeys > kwin_lo) {   // warp has work here
             float sc[8][4];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
@@ -167,11 +179,12 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     mma16816<BF16>(sc[nt], qa[2 * kk + 1], bk[2], bk[3]);
                 }
             }
-            const bool need_mask = key0 + kKeys > kmin_warp;
+            const bool need_mask = key0 + kKeys > kmin_warp || key0 < kwin_hi;
             float alpha[2];
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 const int kmax = hr ? kmax1 : kmax0;
+                const int klo = hr ? klo1 : klo0;
                 float mx = -INFINITY;
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt)
@@ -179,7 +192,7 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                     for (int e = 0; e < 2; ++e) {
                         const int key = key0 + nt * 8 + 2 * qd + e;
                         float x = sc[nt][2 * hr + e] * sl;
-                        if (need_mask && key >= kmax) x = -INFINITY;
+                        if (need_mask && (key >= kmax || key < klo)) x = -INFINITY;
                         sc[nt][2 * hr + e] = x;
                         mx = fmaxf(mx, x);
                     }
@@ -221,12 +234,13 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
                         al[2 * hh + hr] = pack2<BF16>(x0 - back.x, x1 - back.y);
                     }
                 }
-                // V rows past the end of the sequence may hold anything: zero them
+                // V rows past the end of the sequence (or before every window) may hold anything: zero them
                 uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
                 const int kb0 = key0 + 16 * kk + 2 * qd;
-                if (key0 + kKeys > seq_len) {
-                    keep_lo = (kb0 < seq_len ? 0x0000ffffu : 0u) | (kb0 + 1 < seq_len ? 0xffff0000u : 0u);
-                    keep_hi = (kb0 + 8 < seq_len ? 0x0000ffffu : 0u) | (kb0 + 9 < seq_len ? 0xffff0000u : 0u);
+                if (key0 + kKeys > seq_len || key0 < lo_cta) {   // and keys no row of the CTA sees
+                    auto in = [&](int key) { return key < seq_len && key >= lo_cta; };
+                    keep_lo = (in(kb0) ? 0x0000ffffu : 0u) | (in(kb0 + 1) ? 0xffff0000u : 0u);
+                    keep_hi = (in(kb0 + 8) ? 0x0000ffffu : 0u) | (in(kb0 + 9) ? 0xffff0000u : 0u);
                 }
 #pragma unroll
                 for (int np = 0; np < D / 16; ++np) {
@@ -299,6 +313,7 @@ int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorM
     p.G = a.G;
     p.N = a.N;
     p.scale_log2 = a.scale * kLog2e;
+    p.window = a.window;
     const bool bf = a.kv_dtype == PKV_BF16;
     if (a.d == 128) return bf ? launch_prefill_mma<128, true>(p, s, tmk, tmv) : launch_prefill_mma<128, false>(p, s, tmk, tmv);
     if (a.d == 64) return bf ? launch_prefill_mma<64, true>(p, s, tmk, tmv) : launch_prefill_mma<64, false>(p, s, tmk, tmv);

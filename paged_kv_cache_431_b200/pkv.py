@@ -37,7 +37,7 @@ class _PoolDesc(ctypes.Structure):
 
 
 class _DecodeOpts(ctypes.Structure):
-    _fields_ = [("engine", ctypes.c_int32), ("partition_tokens", ctypes.c_int32)]
+    _fields_ = [("engine", ctypes.c_int32), ("partition_tokens", ctypes.c_int32), ("sliding_window", ctypes.c_int32)]
 
 
 _lib = None
@@ -211,34 +211,37 @@ def kv_append(pool: KVPool, layer: int, k: torch.Tensor, v: torch.Tensor, slot_m
                            else 0, _stream(stream)), "kv_append")
 
 
-def _opts(engine: int, partition_tokens: int):
-    if engine == 0 and partition_tokens == 0:
+def _opts(engine: int, partition_tokens: int, sliding_window: int = 0):
+    if engine == 0 and partition_tokens == 0 and sliding_window == 0:
         return None
-    return ctypes.byref(_DecodeOpts(engine, partition_tokens))
+    return ctypes.byref(_DecodeOpts(engine, partition_tokens, sliding_window))
 
 
 def paged_decode_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int, max_context_len: int,
-                                 engine: int = 0, partition_tokens: int = 0) -> int:
+                                 engine: int = 0, partition_tokens: int = 0, sliding_window: int = 0) -> int:
     return int(lib().paged_decode_workspace_bytes(pool.handle, num_seqs, num_q_heads, max_context_len,
-                                                  _opts(engine, partition_tokens)))
+                                                  _opts(engine, partition_tokens, sliding_window)))
 
 
 def paged_decode_attn(pool: KVPool, layer: int, q: torch.Tensor, block_tables: torch.Tensor,
                       context_lens: torch.Tensor, scale: float, max_context_len: int,
                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                      engine: int = 0, partition_tokens: int = 0, stream=None) -> torch.Tensor:
-    """Decode attention for q [B, H_q, head_dim]; returns fp32 out [B, H_q, head_dim]."""
+                      engine: int = 0, partition_tokens: int = 0, sliding_window: int = 0,
+                      stream=None) -> torch.Tensor:
+    """Decode attention for q [B, H_q, head_dim]; returns fp32 out [B, H_q, head_dim].
+    sliding_window > 0: the query sees only the last sliding_window positions."""
     B, H_q, d = q.shape
     if out is None:
         out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
-    need = paged_decode_workspace_bytes(pool, B, H_q, max_context_len, engine, partition_tokens)
+    need = paged_decode_workspace_bytes(pool, B, H_q, max_context_len, engine, partition_tokens, sliding_window)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().paged_decode_attn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_tables),
                                    block_tables.shape[1], _ptr(context_lens), B, H_q, max_context_len,
                                    float(scale), _ptr(out), _ptr(workspace), ws_bytes,
-                                   _opts(engine, partition_tokens), _stream(stream)), "paged_decode_attn")
+                                   _opts(engine, partition_tokens, sliding_window), _stream(stream)),
+           "paged_decode_attn")
     return out
 
 
@@ -256,7 +259,7 @@ def paged_decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, block_t
                               context_lens: torch.Tensor, scale: float, max_context_len: int,
                               shared_prefix_len: int, out: torch.Tensor | None = None,
                               workspace: torch.Tensor | None = None, engine: int = 0, partition_tokens: int = 0,
-                              stream=None) -> torch.Tensor:
+                              sliding_window: int = 0, stream=None) -> torch.Tensor:
     """Decode attention for a batch whose tables all start with the same shared_prefix_len
     tokens (row 0's blocks): the prefix is attended once per KV group on the tensor cores."""
     L = lib()
@@ -274,7 +277,7 @@ def paged_decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, block_t
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_tables), block_tables.shape[1],
               _ptr(context_lens), B, H_q, max_context_len, shared_prefix_len, float(scale), _ptr(out),
-              _ptr(workspace), ws_bytes, _opts(engine, partition_tokens), _stream(stream)),
+              _ptr(workspace), ws_bytes, _opts(engine, partition_tokens, sliding_window), _stream(stream)),
            "paged_decode_attn_cascade")
     return out
 
@@ -285,7 +288,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 def paged_decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, block_tables: torch.Tensor,
                               context_lens: torch.Tensor, scale: float, max_context_len: int,
                               out: torch.Tensor | None = None, engine: int = 0, partition_tokens: int = 0,
-                              stream=None) -> torch.Tensor:
+                              sliding_window: int = 0, stream=None) -> torch.Tensor:
     """paged_decode_attn without a workspace argument, for callers that cannot allocate device
     memory for one: the split-K partials use the library's fixed 32 MiB device buffer.  Only
     the output is the caller's.  Calls that may overlap on the GPU share that buffer and race;
@@ -300,20 +303,30 @@ def paged_decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, block_t
         out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
     _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_tables), block_tables.shape[1],
               _ptr(context_lens), B, H_q, max_context_len, float(scale), _ptr(out),
-              _opts(engine, partition_tokens), _stream(stream)), "paged_decode_attn_noalloc")
+              _opts(engine, partition_tokens, sliding_window), _stream(stream)), "paged_decode_attn_noalloc")
     return out
 
 
 def paged_prefill_chunk_attn(pool: KVPool, layer: int, q: torch.Tensor, block_table: torch.Tensor,
                              ctx_before: int, scale: float, out: torch.Tensor | None = None,
-                             stream=None) -> torch.Tensor:
-    """Chunked-prefill attention for q [C, H_q, head_dim] at positions ctx_before + i."""
+                             sliding_window: int = 0, stream=None) -> torch.Tensor:
+    """Chunked-prefill attention for q [C, H_q, head_dim] at positions ctx_before + i
+    (sliding_window > 0: each row sees only the last sliding_window positions up to itself)."""
     C, H_q, d = q.shape
     if out is None:
         out = torch.empty(C, H_q, d, dtype=torch.float32, device=q.device)
-    _check(lib().paged_prefill_chunk_attn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_table),
-                                          block_table.shape[-1], ctx_before, C, H_q, float(scale), _ptr(out),
-                                          None, 0, _stream(stream)), "paged_prefill_chunk_attn")
+    if sliding_window == 0:
+        _check(lib().paged_prefill_chunk_attn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_table),
+                                              block_table.shape[-1], ctx_before, C, H_q, float(scale), _ptr(out),
+                                              None, 0, _stream(stream)), "paged_prefill_chunk_attn")
+        return out
+    L = lib()
+    fn = L.paged_prefill_chunk_attn_window
+    P, i32 = ctypes.c_void_p, ctypes.c_int
+    fn.restype = i32
+    fn.argtypes = [P, i32, P, i32, P, i32, i32, i32, i32, ctypes.c_float, i32, P, P]
+    _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_table), block_table.shape[-1], ctx_before, C,
+              H_q, float(scale), int(sliding_window), _ptr(out), _stream(stream)), "paged_prefill_chunk_attn_window")
     return out
 
 

@@ -92,8 +92,16 @@ def test_decode_and_append_argument_checks():
     try:
         # H_q not a multiple of H_kv
         assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 3, 64, 0.1, fake, None, 0, None, None) == -4
-        # G = 20 > 16
-        assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 40, 64, 0.1, fake, None, 0, None, None) == -9
+        # a negative sliding window
+        bad = pkv._DecodeOpts(0, 0, -1)
+        assert L.paged_decode_attn(h, 0, fake, pkv.F16, fake, 4, fake, 4, 8, 64, 0.1, fake, None, 0,
+                                   ctypes.byref(bad), None) == -2
+        assert L.paged_decode_workspace_bytes(h, 4, 8, 64, ctypes.byref(bad)) == 0
+        # a window shrinks the split-K grid: 100,000 tokens with a 256-token window need no more
+        # partials than 271 tokens do
+        win = pkv._DecodeOpts(0, 0, 256)
+        assert L.paged_decode_workspace_bytes(h, 4, 8, 100000, ctypes.byref(win)) == \
+            L.paged_decode_workspace_bytes(h, 4, 8, 271, None)
         # q dtype must match a 16-bit pool
         assert L.paged_decode_attn(h, 0, fake, pkv.BF16, fake, 4, fake, 4, 8, 64, 0.1, fake, None, 0, None, None) == -3
         # bad layer
