@@ -155,6 +155,14 @@ WORKLOADS = {
                        lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("packed int4")),
     "quant_bf16": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=8192,
                        lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("bf16 (control)")),
+    "mqa": dict(kind="decode", layers=1, B=256, H_q=64, H_kv=1, d=128, dtype=wl.BF16, width=256,
+                lens="gqa70b", pool_blocks=256 * 256,
+                desc="MQA decode (one KV head for all 64 query heads, G = 64), 1 layer, d 128, bf16, B 256, "
+                     "ctx ~ N(3000, 400) clipped to [1024, 4096]"),
+    "window": dict(kind="decode", layers=1, B=64, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=2048,
+                   lens="long", pool_blocks=64 * 2048, window=4096,
+                   desc="sliding-window decode, 1 layer of the 70B shape (H_q 64, H_kv 8, d 128, bf16), B 64, "
+                        "ctx ~ U[16384, 32768], window 4,096 tokens: only the window's K/V is read"),
     "prefix_chunk": dict(kind="prefix", layers=1, B=256, H_q=64, H_kv=8, d=128, dtype=wl.BF16,
                          desc="prefix sharing + chunked prefill, 1 layer of the 70B shape, bf16: 256 decodes "
                               "share a 4,000-token prefix (250 blocks) + private 200-token suffixes + U{0..300} "
@@ -166,12 +174,17 @@ DTYPE_NAME = {wl.F16: "f16", wl.BF16: "bf16", wl.INT8: "int8", wl.FP8: "fp8e4m3"
 
 
 def make_lens(kind, gen, B):
+    if kind == "long":
+        return torch.randint(16384, 32769, (B,), generator=gen, dtype=torch.int32)
     return {"gqa70b": wl.gqa70b_lens, "llama8b": wl.llama8b_lens, "quant": wl.quant_long_lens}[kind](gen, B)
 
 
-def decode_bytes(ctx_lens, B, H_q, H_kv, d, dt):
-    """(K/V bytes, all algorithmic bytes) of one decode call: every cached K and V
-    element once (and its block's scales), plus q, out, used table entries, lengths."""
+def decode_bytes(ctx_lens, B, H_q, H_kv, d, dt, window=0):
+    """(K/V bytes, all algorithmic bytes) of one decode call: every visible cached K and V
+    element once (and its block's scales), plus q, out, used table entries, lengths.  With a
+    sliding window only the last `window` tokens of each context are visible."""
+    if window:
+        ctx_lens = torch.clamp(ctx_lens, max=window)
     sum_ctx = int(ctx_lens.sum())
     blocks = int(sum(wl.ceil_div(int(n), 16) for n in ctx_lens))
     kv = int(sum_ctx * 2 * H_kv * d * ELEM_BYTES[dt])
@@ -237,7 +250,9 @@ def build_decode(args, cfg, dev, rank):
     k_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     v_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     out = torch.empty(L, B, H_q, d, dtype=torch.float32, device=dev)
-    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition), 16),
+    window = cfg.get("window", 0)
+    ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition,
+                                                          sliding_window=window), 16),
                      dtype=torch.uint8, device=dev)
     aws = torch.empty(max(pkv.kv_append_workspace_bytes(pool, B), 16), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -250,12 +265,12 @@ def build_decode(args, cfg, dev, rank):
             if ev is not None:
                 ev[l][0].record(stream)
             pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws,
-                                  engine=args.engine, partition_tokens=args.partition)
+                                  engine=args.engine, partition_tokens=args.partition, sliding_window=window)
             if ev is not None:
                 ev[l][1].record(stream)
 
-    kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt)
-    parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx) > 0
+    kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt, window)
+    parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, sliding_window=window) > 0
     launches = L * ((3 if quant else 1) + 1 + (1 if parts else 0))
 
     # host-buffer (e2e) step: inputs from pinned memory, every layer's output read back
@@ -294,7 +309,7 @@ def build_decode(args, cfg, dev, rank):
             stream.wait_event(ready[l])
             pkv.kv_append(pool, l % L_phys, dk[l], dv[l], dslots, workspace=aws)
             pkv.paged_decode_attn(pool, l % L_phys, dq[l], dtab, dctx, scale, max_ctx, out=dout[l], workspace=ws,
-                                  engine=args.engine, partition_tokens=args.partition)
+                                  engine=args.engine, partition_tokens=args.partition, sliding_window=window)
             e = torch.cuda.Event()
             e.record(stream)
             done.append(e)
@@ -314,10 +329,11 @@ def build_decode(args, cfg, dev, rank):
                 "kv_heads": H_kv, "head_dim": d, "kv_dtype": DTYPE_NAME[dt], "sum_ctx": int(ctx.sum()),
                 "physical_layer_pools": L_phys, "parallelism": "replicas",
                 "l2": f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V",
-                "partition_tokens": args.partition or "auto",
+                "partition_tokens": args.partition or "auto", "sliding_window": window or None,
                 "decode_engine": {0: "tensor cores (mma.sync)", 1: "tensor cores (mma.sync)",
                                   2: "CUDA cores, packed fp32x2 FMA", 3: "CUDA cores, fp32 FMA"}[args.engine]},
-        kv_bytes_per_step=kv * L, seq_tokens_per_step=int(ctx.sum()) * L, layers=L,
+        kv_bytes_per_step=kv * L, layers=L,
+        seq_tokens_per_step=int((torch.clamp(ctx, max=window) if window else ctx).sum()) * L,
         roofline=dict(bound="hbm", kernel="paged_decode_attn (main + split-K merge)", alg_bytes=alg,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
@@ -433,6 +449,22 @@ def build_prefix_chunk(args, cfg, dev, rank):
     return step, e2e_step, info, pool
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks: the slowest replica bounds the whole job.  The
+    identity without a process group (one GPU)."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step: float, steps: int, world: int, elapsed_ms: float) -> float:
+    """Whole-job units per second: every rank processes units_per_step each step (weak
+    scaling, independent replicas), all ranks within elapsed_ms (the max over ranks)."""
+    return units_per_step * steps * world / (elapsed_ms * 1e-3)
+
+
 def time_steps(step, n_steps, per_step_calls, dev, world):
     timed = Timed(n_steps, per_step_calls)
     stream = torch.cuda.current_stream(dev)
@@ -448,9 +480,8 @@ def time_steps(step, n_steps, per_step_calls, dev, world):
     torch.cuda.synchronize(dev)
     ms = t0.elapsed_time(t1)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        torch.distributed.barrier()
+        ms = max_over_ranks(ms, dev)
     return ms, timed
 
 
@@ -488,8 +519,8 @@ def run_gpu(args):
     e2e_ms, _ = time_steps(lambda ev=None: e2e_step(), args.steps, 1, dev, world)
 
     ms_per_step = elapsed_ms / args.steps
-    value = info["kv_bytes_per_step"] * args.steps * world / (elapsed_ms * 1e-3) / 1e9
-    e2e_value = info["kv_bytes_per_step"] * args.steps * world / (e2e_ms * 1e-3) / 1e9
+    value = job_throughput(info["kv_bytes_per_step"], args.steps, world, elapsed_ms) / 1e9
+    e2e_value = job_throughput(info["kv_bytes_per_step"], args.steps, world, e2e_ms) / 1e9
     call_ms = timed.call_ms()
     rf = info["roofline"]
     if rf["bound"] == "hbm":
@@ -518,8 +549,8 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": info["dtype"], "data": "synthetic",
         "config": info["config"],
-        "seq_tokens_per_s_per_layer": round(info["seq_tokens_per_step"] / info["layers"] * args.steps * world
-                                            / (elapsed_ms * 1e-3)),
+        "seq_tokens_per_s_per_layer": round(job_throughput(info["seq_tokens_per_step"] / info["layers"],
+                                                           args.steps, world, elapsed_ms)),
         "pct_of_8tbs_nominal": round(100 * value / world / 8000.0, 1),
         "roofline": roofline,
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "ms_per_step": round(e2e_ms / args.steps, 4),
@@ -572,11 +603,13 @@ def cpu_oracle(workload, budget_s=12.0, per_step=None, steps=None, warmup=0):
             oracle.kv_append(opool, k, v, oracle.BF16, np.arange(n, dtype=np.int32))
             q = wl.normal((1, H_q, d), torch.bfloat16, gh)
             t0 = time.perf_counter()
-            oracle.paged_decode(opool, q, oracle.BF16, table, [n], np.float32(d ** -0.5))
+            window = cfg.get("window", 0)
+            oracle.paged_decode(opool, q, oracle.BF16, table, [n], np.float32(d ** -0.5), window=window)
             step_s += time.perf_counter() - t0
             if s >= warmup:
-                total_kv += int(n * 2 * H_kv * d * ELEM_BYTES[dt])
-                total_tok += n
+                seen = min(n, window) if window else n
+                total_kv += int(seen * 2 * H_kv * d * ELEM_BYTES[dt])
+                total_tok += seen
                 seqs += 1
         if s >= warmup:
             total_s += step_s

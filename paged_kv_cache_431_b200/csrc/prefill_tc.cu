@@ -168,8 +168,10 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 
 struct Bars {
     uint64_t q_full;
-    uint64_t kv_full[kNS];
-    uint64_t kv_empty[kNS];
+    uint64_t k_full[kNS];      // K and V rings are separate: a K stage frees when its
+    uint64_t k_empty[kNS];     // Q.K^T is done, a V stage when its P.V is done, so the next
+    uint64_t v_full[kNS];      // K tile can land while the previous P.V still reads V
+    uint64_t v_empty[kNS];
     uint64_t s_full[2];
     uint64_t s_free[2];
     uint64_t p_full;
@@ -208,8 +210,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         s_abort = 0;
         mbar_init(smem_u32(&bars.q_full), 1);
         for (int s = 0; s < kNS; ++s) {
-            mbar_init(smem_u32(&bars.kv_full[s]), 1);
-            mbar_init(smem_u32(&bars.kv_empty[s]), 1);
+            mbar_init(smem_u32(&bars.k_full[s]), 1);
+            mbar_init(smem_u32(&bars.k_empty[s]), 1);
+            mbar_init(smem_u32(&bars.v_full[s]), 1);
+            mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&bars.s_full[b]), 1);
@@ -259,38 +263,57 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         }
         int cur = table_entry(lane);                         // chunk 0
         int nxt = table_entry(32 + lane);                    // chunk 1
-        int issued = 0;
+        int issued = 0, issued_k = 0;   // tiles whose V (and K) copies were issued
         for (int t = 0; t < ntiles; ++t) {
             const int s = t % kNS;
             if (t > 0 && t % kTilesPerChunk == 0) {
                 cur = nxt;
                 nxt = table_entry((t / kTilesPerChunk + 1) * 32 + lane);
             }
-            bool go = true;
-            if (lane == 0 && t >= kNS)
-                go = wait_or_abort(smem_u32(&bars.kv_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
-            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
-            const uint32_t fb = smem_u32(&bars.kv_full[s]);
-            if (lane == 0) mbar_arrive_expect_tx(fb, 2 * kKVBytes);
+            int blk_of[kBlkPerTile];
 #pragma unroll
             for (int kb = 0; kb < kBlkPerTile; ++kb) {
                 const int blk = __shfl_sync(0xffffffffu, cur, (t % kTilesPerChunk) * kBlkPerTile + kb);
                 // past the sequence: block 0 (in bounds; those keys are masked and their V zeroed)
-                const int row = ((blk < 0 ? 0 : blk) * p.H_kv + g) * kBlock;
-                if (lane == 0) {
-#pragma unroll
-                    for (int x = 0; x < 2; ++x) {
-                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, row, fb);
-                        tma_load_2d(sV + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmV, 64 * x, row, fb);
-                    }
-                }
+                blk_of[kb] = ((blk < 0 ? 0 : blk) * p.H_kv + g) * kBlock;
             }
+            bool go = true;
+            if (lane == 0 && t >= kNS)
+                go = wait_or_abort(smem_u32(&bars.k_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
+            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
+            if (lane == 0) {
+                const uint32_t fb = smem_u32(&bars.k_full[s]);
+                mbar_arrive_expect_tx(fb, kKVBytes);
+#pragma unroll
+                for (int kb = 0; kb < kBlkPerTile; ++kb)
+#pragma unroll
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, blk_of[kb], fb);
+            }
+            if (lane == 0 && t >= kNS)
+                go = wait_or_abort(smem_u32(&bars.v_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
+            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) {
+                issued_k = t + 1;
+                break;
+            }
+            if (lane == 0) {
+                const uint32_t fb = smem_u32(&bars.v_full[s]);
+                mbar_arrive_expect_tx(fb, kKVBytes);
+#pragma unroll
+                for (int kb = 0; kb < kBlkPerTile; ++kb)
+#pragma unroll
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_2d(sV + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmV, 64 * x, blk_of[kb], fb);
+            }
+            issued_k = t + 1;
             issued = t + 1;
         }
         // do not leave while copies into this CTA's shared memory may be in flight
         if (lane == 0 && s_abort) {
+            for (int t = max(0, issued_k - kNS); t < issued_k; ++t)
+                mbar_wait_bounded(smem_u32(&bars.k_full[t % kNS]), (t / kNS) & 1);
             for (int t = max(0, issued - kNS); t < issued; ++t)
-                mbar_wait_bounded(smem_u32(&bars.kv_full[t % kNS]), (t / kNS) & 1);
+                mbar_wait_bounded(smem_u32(&bars.v_full[t % kNS]), (t / kNS) & 1);
             mbar_wait_bounded(qb, 0);
         }
     } else if (warp == 1) {
@@ -302,7 +325,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             for (int t = 0; ok && t <= ntiles; ++t) {
                 if (t < ntiles) {
                     const int s = t % kNS, b = t & 1;
-                    if (!wait_or_abort(smem_u32(&bars.kv_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
+                    if (!wait_or_abort(smem_u32(&bars.k_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
                     if (t >= 2 && !wait_or_abort(smem_u32(&bars.s_free[b]), ((t - 2) >> 1) & 1, &s_abort, p.status))
                         break;
                     tc_fence_after();
@@ -313,10 +336,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                         umma(tmem + b * kBN, sdesc_k128(sQ + off), sdesc_k128(kbase + off), id_qk, ks > 0);
                     }
                     umma_commit(smem_u32(&bars.s_full[b]));
+                    umma_commit(smem_u32(&bars.k_empty[s]));
                 }
                 if (t >= 1) {
                     const int u = t - 1, s = u % kNS;
                     if (!wait_or_abort(smem_u32(&bars.p_full), u & 1, &s_abort, p.status)) break;
+                    if (!wait_or_abort(smem_u32(&bars.v_full[s]), (u / kNS) & 1, &s_abort, p.status)) break;
                     tc_fence_after();
                     const uint32_t vbase = sV + s * kKVBytes;
 #pragma unroll
@@ -327,7 +352,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                         umma(tmem + 2 * kBN, sdesc_k128(sPl + poff), bv, id_pv, true);
                     }
                     umma_commit(smem_u32(&bars.o_done));
-                    umma_commit(smem_u32(&bars.kv_empty[s]));
+                    umma_commit(smem_u32(&bars.v_empty[s]));
                 }
             }
         }
@@ -468,7 +493,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             // keys past the end of the sequence: zero their V rows (P is 0 there, V may be stale)
             if (t == ntiles - 1 && t * kBN + kBN > seq_len) {
                 const int s = t % kNS;
-                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.kv_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
+                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
                     ok = false;
                     break;
                 }
