@@ -46,7 +46,7 @@ METRIC = "paged GQA decode: KV HBM GB/s (% of ~8 TB/s peak); seq-tokens/s per la
 PROFILES = os.path.join(ROOT, "profiles")
 DECODE_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_quant.cu",
                "paged_kv_cache_431_b200/csrc/decode_common.cuh", "paged_kv_cache_431_b200/csrc/common.cuh"]
-PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
+PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
 
 
 # ------------------------------------------------------------------ utils --
@@ -155,6 +155,10 @@ WORKLOADS = {
                        lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("packed int4")),
     "quant_bf16": dict(kind="decode", layers=1, B=16, H_q=64, H_kv=8, d=128, dtype=wl.BF16, width=8192,
                        lens="quant", pool_blocks=16 * 8192, desc=QUANT_DESC.format("bf16 (control)")),
+    "mha": dict(kind="decode", layers=1, B=32, H_q=64, H_kv=64, d=128, dtype=wl.BF16, width=256,
+                lens="gqa70b", pool_blocks=32 * 256,
+                desc="MHA decode (one KV head per query head, G = 1), 1 layer, H 64, d 128, bf16, B 32, "
+                     "ctx ~ N(3000, 400) clipped to [1024, 4096]"),
     "mqa": dict(kind="decode", layers=1, B=256, H_q=64, H_kv=1, d=128, dtype=wl.BF16, width=256,
                 lens="gqa70b", pool_blocks=256 * 256,
                 desc="MQA decode (one KV head for all 64 query heads, G = 64), 1 layer, d 128, bf16, B 256, "

@@ -95,7 +95,7 @@ int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtenso
 // dtype (512 tokens for bf16 at head_dim 128, 1024 for int8 / fp8, 2048 for int4), so the
 // partials stay near 1.6% of the bytes read; smaller (down to 128 tokens) when the batch
 // is too small to fill the GPU with one-warp CTAs.
-static int choose_partition(int B, int H_kv, int max_ctx, int row_bytes, const pkv_decode_opts* o)
+static int choose_partition(int B, int ctas, int max_ctx, int row_bytes, const pkv_decode_opts* o)
 {
     if (o && o->partition_tokens > 0) return o->partition_tokens;
     int P = 256 * 1024 / (2 * row_bytes);
@@ -103,7 +103,7 @@ static int choose_partition(int B, int H_kv, int max_ctx, int row_bytes, const p
     const long target = 4L * num_sms() * 8;
     while (P > 128) {
         const long parts = (max_ctx + P - 1) / P;
-        if ((long)B * H_kv * (parts > 0 ? parts : 1) >= target) break;
+        if ((long)B * ctas * (parts > 0 ? parts : 1) >= target) break;
         P /= 2;
     }
     return P;
@@ -228,14 +228,22 @@ int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, int src_
     return launch_append(a, static_cast<cudaStream_t>(stream));
 }
 
-static int decode_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, const pkv_decode_opts* opts, int* P,
-                               int* max_parts)
+// CTAs the decode grid has per (sequence, partition): one per KV head and group of 16 query heads.
+static int ctas_per_partition(pkv_pool_t pool, int num_q_heads)
+{
+    const int H_kv = pool->d.num_kv_heads;
+    const int G = (num_q_heads > 0 && num_q_heads % H_kv == 0) ? num_q_heads / H_kv : 1;
+    return H_kv * ((G + 15) / 16);
+}
+
+static int decode_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_ctx,
+                               const pkv_decode_opts* opts, int* P, int* max_parts)
 {
     const int window = opts ? opts->sliding_window : 0;
     if (window < 0) return PKV_ERR_ARG;
     // with a window a sequence's partitions start at the block holding ctx - window
     const int span = (window > 0 && max_ctx > window + PKV_BLOCK_SIZE - 1) ? window + PKV_BLOCK_SIZE - 1 : max_ctx;
-    *P = choose_partition(num_seqs, pool->d.num_kv_heads, span, pool->row_bytes, opts);
+    *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), span, pool->row_bytes, opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
     *max_parts = span > 0 ? (span + *P - 1) / *P : 1;
     return PKV_OK;
@@ -246,7 +254,7 @@ size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_hea
 {
     if (!pool || num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return 0;
     int P, parts;
-    if (decode_partitioning(pool, num_seqs, max_context_len, opts, &P, &parts) != PKV_OK) return 0;
+    if (decode_partitioning(pool, num_seqs, num_q_heads, max_context_len, opts, &P, &parts) != PKV_OK) return 0;
     if (parts <= 1) return 0;
     return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float);
 }
@@ -273,7 +281,7 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     if (engine < 0 || engine > 3) return PKV_ERR_ARG;
     if (engine == 0) engine = 1;
     int P, parts;
-    int rc = decode_partitioning(pool, num_seqs, max_context_len, opts, &P, &parts);
+    int rc = decode_partitioning(pool, num_seqs, num_q_heads, max_context_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;
     const size_t need = parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (d.head_dim + 2) * sizeof(float) : 0;
     if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15)))
@@ -321,11 +329,12 @@ static bool cascade_shape_ok(pkv_pool_t pool, int num_q_heads, int max_context_l
            max_context_len >= prefix_len;
 }
 
-static int cascade_partitioning(pkv_pool_t pool, int num_seqs, int max_ctx, int prefix_len,
+static int cascade_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_ctx, int prefix_len,
                                 const pkv_decode_opts* opts, int* P, int* suffix_parts)
 {
     const int rest = max_ctx - prefix_len;
-    *P = choose_partition(num_seqs, pool->d.num_kv_heads, rest > 0 ? rest : 1, pool->row_bytes, opts);
+    *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), rest > 0 ? rest : 1, pool->row_bytes,
+                          opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
     *suffix_parts = rest > 0 ? (rest + *P - 1) / *P : 1;
     return PKV_OK;
@@ -338,7 +347,9 @@ size_t paged_decode_cascade_workspace_bytes(pkv_pool_t pool, int num_seqs, int n
     if (shared_prefix_len == 0) return paged_decode_workspace_bytes(pool, num_seqs, num_q_heads, max_context_len, opts);
     if (!cascade_shape_ok(pool, num_q_heads, max_context_len, shared_prefix_len)) return 0;
     int P, parts;
-    if (cascade_partitioning(pool, num_seqs, max_context_len, shared_prefix_len, opts, &P, &parts) != PKV_OK) return 0;
+    if (cascade_partitioning(pool, num_seqs, num_q_heads, max_context_len, shared_prefix_len, opts, &P, &parts) !=
+        PKV_OK)
+        return 0;
     return (size_t)num_seqs * num_q_heads * (1 + parts) * (pool->d.head_dim + 2) * sizeof(float);
 }
 
@@ -370,7 +381,7 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     if (engine < 0 || engine > 3) return PKV_ERR_ARG;
     if (engine == 0) engine = 1;
     int P, parts;
-    int rc = cascade_partitioning(pool, num_seqs, max_context_len, shared_prefix_len, opts, &P, &parts);
+    int rc = cascade_partitioning(pool, num_seqs, num_q_heads, max_context_len, shared_prefix_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;
     const int slots = 1 + parts;
     const size_t need = (size_t)num_seqs * num_q_heads * slots * (d.head_dim + 2) * sizeof(float);

@@ -5,24 +5,26 @@
 // chunk of C positions P0 .. P0+C-1 attends causally to the paged context (possibly a
 // shared prefix, section "Prefix caching") and to itself.
 //
-// One CTA owns 128 query rows of one KV group -- 128/G positions x its G heads -- and
-// walks the keys in tiles of 128 (8 paged blocks):
-//   warp 0      TMA producer: Q once (a 3-D box over [position][head][dim]), then the
-//               K and V tiles of each step block by block through the pool's tensor
-//               maps into a 2-stage ring (128-byte swizzle, no multicast);
-//   warp 1      allocates 512 TMEM columns and issues the MMAs from one thread:
-//               S_t = Q . K_t^T into one of two TMEM score buffers (M=128, N=128, K=16
-//               per instruction), then O += P_{t-1} . V_{t-1} into the TMEM output
-//               accumulator, so the score MMA of a tile overlaps the softmax of the
-//               previous one;
-//   warps 2..9  softmax, two threads per query row (= TMEM lane), each with half the
-//               keys of a tile and half the output dims: read the score row
-//               from TMEM, mask (causal bound P0 + position, end of sequence), keep the
-//               running max lazily (it moves only when the new max exceeds the old by 2^8,
-//               and then O is rescaled in TMEM), write P as a high and a low bf16/f16 part
-//               into shared memory (two MMAs keep P . V at ~16 mantissa bits), and finally
-//               read O, divide by the row sum and store fp32 rows.
-// Every wait is bounded; a timeout sets PKV_DEV_TIMEOUT and the CTA winds down.
+// One CTA owns two query tiles A and B of 128 rows each -- 256/G positions x the G heads of
+// one KV group -- and walks the keys in tiles of 128 (8 paged blocks) shared by both:
+//   warp 0      TMA producer: Q once (3-D boxes over [position][head][dim]), then K and V
+//               tiles block by block through the pool's tensor maps into separate 2-stage
+//               rings (128-byte swizzle, no multicast): a K stage is free once its Q.K^T is
+//               done, a V stage once its P.V is done;
+//   warp 1      allocates all 512 TMEM columns -- per query tile 128 for S (later P) and
+//               128 for the O accumulator -- and issues every MMA from one thread;
+//   warps 2..5  softmax of tile A, warps 6..9 of tile B, one thread per query row (= TMEM
+//               lane): read the row's 128 scores, mask (causal bound, window, end of
+//               sequence), keep the running max lazily (it moves only when the new max
+//               exceeds the old by 2^8, then O is rescaled in TMEM), and write P back into
+//               the score's own TMEM columns as a high and a low 16-bit part (two MMAs keep
+//               P . V at ~16 mantissa bits), where the P . V MMA reads it as its A operand.
+// The two tiles ping-pong: while the softmax warps of one tile work, the tensor cores run
+// the other tile's P . V and next Q.K^T, so neither unit waits for the other:
+//   MMA order per key tile t:  P.V(A, t), Q.K^T(A, t+1), P.V(B, t), Q.K^T(B, t+1).
+// Tensor-core instructions issued by one thread execute in order, so Q.K^T(A, t+1) may
+// overwrite the columns P.V(A, t) reads.  Every wait is bounded; a timeout sets
+// PKV_DEV_TIMEOUT and the CTA winds down.
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,15 +33,15 @@ namespace pkv {
 namespace {
 
 constexpr int kD = 128;             // head dim handled here
-constexpr int kBM = 128;            // query rows per CTA
+constexpr int kBM = 128;            // query rows per tile
+constexpr int kQT = 2;              // query tiles per CTA
 constexpr int kBN = 128;            // keys per tile
-constexpr int kNS = 2;              // K/V ring stages
-constexpr int kQBytes = kBM * kD * 2;            // 32 KiB
-constexpr int kKVBytes = kBN * kD * 2;           // 32 KiB each for K and V
-constexpr int kPBytes = kBM * kBN * 2;           // 32 KiB each for P hi and P lo
-constexpr int kSmem = kQBytes + kNS * 2 * kKVBytes + 2 * kPBytes + 1024;
-constexpr uint32_t kTmemCols = 512;              // S0, S1, O (128 columns each)
-constexpr int kThreads = 320;                    // producer, MMA, 8 softmax warps
+constexpr int kNS = 2;              // stages of each of the K and V rings
+constexpr int kQBytes = kBM * kD * 2;            // 32 KiB per query tile
+constexpr int kKVBytes = kBN * kD * 2;           // 32 KiB per K (or V) stage
+constexpr int kSmem = kQT * kQBytes + kNS * 2 * kKVBytes + 1024;
+constexpr uint32_t kTmemCols = 512;              // tile x: S/P at 256x, O at 256x + 128
+constexpr int kThreads = 320;                    // producer, MMA, 2 x 4 softmax warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.f;             // log2 units
 
@@ -90,6 +92,17 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, ui
         : "memory");
 }
 
+// D (TMEM) += A (TMEM) . B (shared memory descriptor)
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -132,16 +145,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
         : "memory");
 }
 
-__device__ __forceinline__ float tmem_ld1(uint32_t taddr)
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32])
 {
-    uint32_t r;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-    return __uint_as_float(r);
-}
-
-__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v)
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -168,15 +181,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 
 struct Bars {
     uint64_t q_full;
-    uint64_t k_full[kNS];      // K and V rings are separate: a K stage frees when its
-    uint64_t k_empty[kNS];     // Q.K^T is done, a V stage when its P.V is done, so the next
-    uint64_t v_full[kNS];      // K tile can land while the previous P.V still reads V
+    uint64_t k_full[kNS];
+    uint64_t k_empty[kNS];
+    uint64_t v_full[kNS];
     uint64_t v_empty[kNS];
-    uint64_t s_full[2];
-    uint64_t s_free[2];
-    uint64_t p_full;
-    uint64_t o_done;
-    uint64_t pair[4];          // the two softmax warps of a TMEM lane quarter
+    uint64_t s_full[kQT];      // S(x, t) is in TMEM (every earlier MMA of the CTA is done too)
+    uint64_t p_full[kQT];      // P(x, t) stored by the four softmax warps of tile x
+    uint64_t o_done[kQT];      // the last P . V of tile x is done
 };
 
 template <bool BF16>
@@ -191,20 +202,18 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.y;
-    const int pos_per_cta = kBM / p.G;
-    const int i0 = blockIdx.x * pos_per_cta;                 // first chunk position of this CTA
-    const int i_end = min(p.C, i0 + pos_per_cta);
+    const int pos_per_tile = kBM / p.G;
+    const int i0 = blockIdx.x * kQT * pos_per_tile;          // first chunk position of this CTA
+    const int i_end = min(p.C, i0 + kQT * pos_per_tile);
     const int seq_len = p.cascade ? p.nkeys : p.P0 + p.C;
     const int kend = p.cascade ? p.nkeys : p.P0 + i_end;     // exclusive key bound of the CTA's last row
     const int ntiles = (kend + kBN - 1) / kBN;
     const int nblk_seq = (seq_len + kBlock - 1) / kBlock;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    const uint32_t sQ = smem_u32(smem);
-    const uint32_t sK = sQ + kQBytes;                        // kNS stages of K
+    const uint32_t sQ = smem_u32(smem);                      // kQT query tiles
+    const uint32_t sK = sQ + kQT * kQBytes;                  // kNS stages of K
     const uint32_t sV = sK + kNS * kKVBytes;                 // kNS stages of V
-    const uint32_t sPh = sV + kNS * kKVBytes;
-    const uint32_t sPl = sPh + kPBytes;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -215,16 +224,14 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             mbar_init(smem_u32(&bars.v_full[s]), 1);
             mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&bars.s_full[b]), 1);
-            mbar_init(smem_u32(&bars.s_free[b]), 8);
+        for (int x = 0; x < kQT; ++x) {
+            mbar_init(smem_u32(&bars.s_full[x]), 1);
+            mbar_init(smem_u32(&bars.p_full[x]), 4);
+            mbar_init(smem_u32(&bars.o_done[x]), 1);
         }
-        mbar_init(smem_u32(&bars.p_full), 8);
-        for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars.pair[q]), 2);
-        mbar_init(smem_u32(&bars.o_done), 1);
         mbar_fence_init();
     }
-    if (warp == 1) {   // TMEM: S0 [0,128), S1 [128,256), O [256,384)
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem_base)),
                      "r"(kTmemCols)
                      : "memory");
@@ -239,8 +246,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         // ------------------------------------------------------------ producer
         // The whole warp walks the tiles: its 32 lanes hold the block ids of the next 4
         // tiles (one coalesced load per 4 tiles, fetched a chunk ahead), lane 0 issues the
-        // copies.  Reading the table one entry at a time between copies would put a global
-        // load latency in front of every block.
+        // copies.
         constexpr int kBlkPerTile = kBN / kBlock;            // 8
         constexpr int kTilesPerChunk = 32 / kBlkPerTile;     // 4
         auto table_entry = [&](int lb) -> int {             // physical block of logical block lb
@@ -257,25 +263,27 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
-            mbar_arrive_expect_tx(qb, kQBytes);
-            tma_load_3d(sQ, &tmQ, 0, g * p.G, i0, qb);
-            tma_load_3d(sQ + kQBytes / 2, &tmQ, 64, g * p.G, i0, qb);
+            mbar_arrive_expect_tx(qb, kQT * kQBytes);
+            for (int x = 0; x < kQT; ++x) {
+                tma_load_3d(sQ + x * kQBytes, &tmQ, 0, g * p.G, i0 + x * pos_per_tile, qb);
+                tma_load_3d(sQ + x * kQBytes + kQBytes / 2, &tmQ, 64, g * p.G, i0 + x * pos_per_tile, qb);
+            }
         }
         int cur = table_entry(lane);                         // chunk 0
         int nxt = table_entry(32 + lane);                    // chunk 1
-        int issued = 0, issued_k = 0;   // tiles whose V (and K) copies were issued
+        int issued = 0, issued_k = 0;                        // tiles whose V (K) copies were issued
         for (int t = 0; t < ntiles; ++t) {
             const int s = t % kNS;
             if (t > 0 && t % kTilesPerChunk == 0) {
                 cur = nxt;
                 nxt = table_entry((t / kTilesPerChunk + 1) * 32 + lane);
             }
-            int blk_of[kBlkPerTile];
+            int row_of[kBlkPerTile];
 #pragma unroll
             for (int kb = 0; kb < kBlkPerTile; ++kb) {
                 const int blk = __shfl_sync(0xffffffffu, cur, (t % kTilesPerChunk) * kBlkPerTile + kb);
                 // past the sequence: block 0 (in bounds; those keys are masked and their V zeroed)
-                blk_of[kb] = ((blk < 0 ? 0 : blk) * p.H_kv + g) * kBlock;
+                row_of[kb] = ((blk < 0 ? 0 : blk) * p.H_kv + g) * kBlock;
             }
             bool go = true;
             if (lane == 0 && t >= kNS)
@@ -288,14 +296,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 for (int kb = 0; kb < kBlkPerTile; ++kb)
 #pragma unroll
                     for (int x = 0; x < 2; ++x)
-                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, blk_of[kb], fb);
+                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, row_of[kb], fb);
             }
+            issued_k = t + 1;
             if (lane == 0 && t >= kNS)
                 go = wait_or_abort(smem_u32(&bars.v_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
-            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) {
-                issued_k = t + 1;
-                break;
-            }
+            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&bars.v_full[s]);
                 mbar_arrive_expect_tx(fb, kKVBytes);
@@ -303,9 +309,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 for (int kb = 0; kb < kBlkPerTile; ++kb)
 #pragma unroll
                     for (int x = 0; x < 2; ++x)
-                        tma_load_2d(sV + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmV, 64 * x, blk_of[kb], fb);
+                        tma_load_2d(sV + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmV, 64 * x, row_of[kb], fb);
             }
-            issued_k = t + 1;
             issued = t + 1;
         }
         // do not leave while copies into this CTA's shared memory may be in flight
@@ -321,209 +326,197 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         if (lane == 0) {
             const uint32_t id_qk = idesc_f16(BF16, false, kBM, kBN);
             const uint32_t id_pv = idesc_f16(BF16, true, kBM, kD);
-            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status);
-            for (int t = 0; ok && t <= ntiles; ++t) {
-                if (t < ntiles) {
-                    const int s = t % kNS, b = t & 1;
-                    if (!wait_or_abort(smem_u32(&bars.k_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
-                    if (t >= 2 && !wait_or_abort(smem_u32(&bars.s_free[b]), ((t - 2) >> 1) & 1, &s_abort, p.status))
-                        break;
-                    tc_fence_after();
-                    const uint32_t kbase = sK + s * kKVBytes;
+            // S(x) = Q(x) . K^T of stage s: M = 128 rows, N = 128 keys, 8 steps of K = 16 dims
+            auto qk = [&](int x, int s) {
+                const uint32_t kbase = sK + s * kKVBytes, qbase = sQ + x * kQBytes;
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32;
-                        umma(tmem + b * kBN, sdesc_k128(sQ + off), sdesc_k128(kbase + off), id_qk, ks > 0);
-                    }
-                    umma_commit(smem_u32(&bars.s_full[b]));
-                    umma_commit(smem_u32(&bars.k_empty[s]));
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32;
+                    umma(tmem + 256 * x, sdesc_k128(qbase + off), sdesc_k128(kbase + off), id_qk, ks > 0);
                 }
-                if (t >= 1) {
-                    const int u = t - 1, s = u % kNS;
-                    if (!wait_or_abort(smem_u32(&bars.p_full), u & 1, &s_abort, p.status)) break;
-                    if (!wait_or_abort(smem_u32(&bars.v_full[s]), (u / kNS) & 1, &s_abort, p.status)) break;
-                    tc_fence_after();
-                    const uint32_t vbase = sV + s * kKVBytes;
+            };
+            // O(x) += P(x) . V of stage s: A = P from TMEM (per 32 keys: 16 columns of high
+            // parts, then 16 of low parts), B = V as an MN-major operand; 8 steps of 16 keys
+            auto pv = [&](int x, int s, bool first) {
+                const uint32_t vbase = sV + s * kKVBytes;
 #pragma unroll
-                    for (int ks = 0; ks < kBN / 16; ++ks) {
-                        const uint32_t poff = (ks >> 2) * (kPBytes / 2) + (ks & 3) * 32;
-                        const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBytes / 2);
-                        umma(tmem + 2 * kBN, sdesc_k128(sPh + poff), bv, id_pv, u > 0 || ks > 0);
-                        umma(tmem + 2 * kBN, sdesc_k128(sPl + poff), bv, id_pv, true);
-                    }
-                    umma_commit(smem_u32(&bars.o_done));
-                    umma_commit(smem_u32(&bars.v_empty[s]));
+                for (int ks = 0; ks < kBN / 16; ++ks) {
+                    const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBytes / 2);
+                    const uint32_t a = tmem + 256 * x + 32 * (ks >> 1) + 8 * (ks & 1);
+                    umma_ts(tmem + 256 * x + 128, a, bv, id_pv, !(first && ks == 0));
+                    umma_ts(tmem + 256 * x + 128, a + 16, bv, id_pv, true);
+                }
+            };
+            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status) &&
+                      wait_or_abort(smem_u32(&bars.k_full[0]), 0, &s_abort, p.status);
+            if (ok) {
+                tc_fence_after();
+                qk(0, 0);
+                umma_commit(smem_u32(&bars.s_full[0]));
+                qk(1, 0);
+                umma_commit(smem_u32(&bars.s_full[1]));
+                umma_commit(smem_u32(&bars.k_empty[0]));
+            }
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int s = t % kNS, s1 = (t + 1) % kNS;
+                const bool more = t + 1 < ntiles;
+                // tile A: P . V, then its next scores
+                if (!wait_or_abort(smem_u32(&bars.p_full[0]), t & 1, &s_abort, p.status)) break;
+                if (!wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
+                tc_fence_after();
+                pv(0, s, t == 0);
+                if (more) {
+                    if (!wait_or_abort(smem_u32(&bars.k_full[s1]), ((t + 1) / kNS) & 1, &s_abort, p.status)) break;
+                    tc_fence_after();
+                    qk(0, s1);
+                    umma_commit(smem_u32(&bars.s_full[0]));
+                } else {
+                    umma_commit(smem_u32(&bars.o_done[0]));
+                }
+                // tile B
+                if (!wait_or_abort(smem_u32(&bars.p_full[1]), t & 1, &s_abort, p.status)) break;
+                tc_fence_after();
+                pv(1, s, t == 0);
+                umma_commit(smem_u32(&bars.v_empty[s]));
+                if (more) {
+                    qk(1, s1);
+                    umma_commit(smem_u32(&bars.s_full[1]));
+                    umma_commit(smem_u32(&bars.k_empty[s1]));
+                } else {
+                    umma_commit(smem_u32(&bars.o_done[1]));
                 }
             }
         }
     } else {
         // ------------------------------------------------------------ softmax
-        // Warps 2..9.  quarter = warp % 4 fixes the 32 TMEM lanes (query rows) a warp may
-        // read; the two warps of a quarter split every row: hc = 0 takes keys 0-63 of a tile
-        // and output dims 0-63, hc = 1 the upper halves.  They combine their row maxima (and,
-        // at the end, their row sums) through spare TMEM columns, ordered by a 2-arrival
-        // mbarrier per quarter.
+        // Warps 2..5: tile A, warps 6..9: tile B.  quarter = warp % 4 fixes the 32 TMEM lanes
+        // (query rows) a warp may touch; one thread per row.
+        const int x = (warp - 2) >> 2;
         const int quarter = warp & 3;
-        const int hc = (warp - 2) >> 2;
-        const int r = quarter * 32 + lane;                   // query row of this thread
-        const int pos = i0 + r / p.G;
-        const int kmax = p.cascade ? p.nkeys : p.P0 + min(pos, p.C - 1) + 1;   // keys < kmax are visible
-        const int kmin_cta = p.cascade ? p.nkeys : p.P0 + i0 + 1;
-        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t xcol = trow + 3 * kBN;                // exchange columns 384..387
-        const uint32_t pair_bar = smem_u32(&bars.pair[quarter]);
+        const int r = quarter * 32 + lane;                   // query row of this thread in tile x
+        const int tile_pos0 = i0 + x * pos_per_tile;
+        const int pos = tile_pos0 + r / p.G;
+        const int kmax = p.cascade ? p.nkeys : p.P0 + min(pos, p.C - 1) + 1;              // keys < kmax visible
+        const int kmin_tile = p.cascade ? p.nkeys : p.P0 + min(tile_pos0, p.C - 1) + 1;   // smallest kmax of tile x
+        const uint32_t tS = tmem + ((uint32_t)(quarter * 32) << 16) + 256 * x;
+        const uint32_t tO = tS + 128;
         const float sl = p.scale_log2;
         const bool pos_scale = sl > 0.f;
         const float slx = pos_scale ? sl : 1.f;              // scale applied inside the exponent
-        float m_used = -INFINITY, l_half = 0.f;
+        float m_used = -INFINITY, l_run = 0.f;
         bool ok = true;
-        // exchange one value per row with the other warp of the quarter; `phase` counts uses
-        auto exchange = [&](float mine, int phase) -> float {
-            const uint32_t slot = xcol + (phase & 1) * 2;
-            tmem_st1(slot + hc, mine);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pair_bar);
-            if (!__all_sync(0xffffffffu, wait_or_abort(pair_bar, phase & 1, &s_abort, p.status))) {
-                ok = false;
-                return mine;
-            }
-            tc_fence_after();
-            const float other = tmem_ld1(slot + (hc ^ 1));
-            tmem_wait_ld();
-            return other;
-        };
         for (int t = 0; t < ntiles; ++t) {
-            const int b = t & 1;
-            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[b]), (t >> 1) & 1, &s_abort, p.status))) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[x]), t & 1, &s_abort, p.status))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            float x[kBN / 2];
-            tmem_ld32(trow + b * kBN + (kBN / 2) * hc, *reinterpret_cast<float(*)[32]>(&x[0]));
-            tmem_ld32(trow + b * kBN + (kBN / 2) * hc + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars.s_free[b]));
-
-            const int key0 = t * kBN + (kBN / 2) * hc;
-            const bool need_mask = t * kBN + kBN > kmin_cta;
+            // pass 1: the row maximum over the tile's 128 scores (64 at a time)
+            const int key0 = t * kBN;
+            const bool need_mask = key0 + kBN > kmin_tile;
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
-            if (pos_scale) {        // max of the raw scores, scaled once
 #pragma unroll
-                for (int j = 0; j < kBN / 2; ++j) {
-                    if (need_mask && key0 + j >= kmax) x[j] = -INFINITY;
-                    m4[j & 3] = fmaxf(m4[j & 3], x[j]);
-                }
-            } else {
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                tmem_ld32(tS + 64 * hh, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+                tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < kBN / 2; ++j) {
-                    x[j] = (need_mask && key0 + j >= kmax) ? -INFINITY : x[j] * sl;
-                    m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+                for (int j = 0; j < 64; ++j) {
+                    const float xj = (need_mask && key0 + 64 * hh + j >= kmax) ? -INFINITY : v[j];
+                    m4[j & 3] = fmaxf(m4[j & 3], pos_scale ? xj : xj * sl);
                 }
             }
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             if (pos_scale) mx *= sl;
-            mx = fmaxf(mx, exchange(mx, t));
-            if (!ok) break;
             float m_new = m_used;
             if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
             const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
-
-            // P = 2^(score - m) as high + low 16-bit parts, computed before waiting for the
-            // previous P . V so the exponentials overlap the tensor cores.  bf16: the high part
-            // is the truncation (upper half of the fp32 word), the low part the truncated
-            // remainder; both are byte permutes, so no conversion instruction is issued.
+            // P = 2^(score - m) as high + low 16-bit parts, back into the score's columns:
+            // keys 32c .. 32c+31 -> columns 32c .. 32c+15 (high), 32c+16 .. 32c+31 (low).
+            // bf16: the high part is the truncation (upper half of the fp32 word), the low part
+            // the truncated remainder, both by byte permutes.
+            // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             float sum = 0.f;
-            uint32_t ph[kBN / 4], pl[kBN / 4];
-#pragma unroll
-            for (int e = 0; e < kBN / 4; ++e) {
-                const float a0 = fmaf(x[2 * e], slx, -mref), a1 = fmaf(x[2 * e + 1], slx, -mref);
-                const float p0 = ex2(a0), p1 = ex2(a1);
-                if constexpr (BF16) {
-                    const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
-                    ph[e] = __byte_perm(u0, u1, 0x7632);
-                    const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
-                    const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-                    pl[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
-                } else {
-                    ph[e] = pack2<false>(p0, p1);
-                    const float2 back = unpack2<false>(ph[e]);
-                    pl[e] = pack2<false>(p0 - back.x, p1 - back.y);
-                }
-                sum += p0 + p1;
-            }
-            if (t > 0) {   // P . V of the previous tile done: P buffers free, O settled
-                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (t - 1) & 1, &s_abort, p.status))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                    for (int c = 0; c < kD / 64; ++c) {
-                        float o[32];
-                        const uint32_t oc = trow + 2 * kBN + (kD / 2) * hc + 32 * c;
-                        tmem_ld32(oc, o);
-                        tmem_wait_ld();
+            for (int c = 0; c < kBN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tS + 32 * c, v);
+                tmem_wait_ld();
+                if (need_mask) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(oc, o);
+                    for (int j = 0; j < 32; ++j)
+                        if (key0 + 32 * c + j >= kmax) v[j] = -INFINITY;
+                }
+                uint32_t w[32];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(v[2 * e], slx, -mref));
+                    const float p1 = ex2(fmaf(v[2 * e + 1], slx, -mref));
+                    if constexpr (BF16) {
+                        const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                        w[e] = __byte_perm(u0, u1, 0x7632);
+                        const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
+                        const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
+                        w[16 + e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                    } else {
+                        w[e] = pack2<false>(p0, p1);
+                        const float2 back = unpack2<false>(w[e]);
+                        w[16 + e] = pack2<false>(p0 - back.x, p1 - back.y);
                     }
-                    tmem_wait_st();
+                    sum += p0 + p1;
+                }
+                tmem_st32u(tS + 32 * c, w);
+            }
+            l_run = l_run * alpha + sum;
+            m_used = m_new;
+            // the running max moved: rescale this row of O (P . V(t-1) is done: s_full(t) says so)
+            if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < kD / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tO + 32 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(tO + 32 * c, o);
                 }
             }
-            // this warp's 64 keys are box hc of P: K-major rows with the 128-byte swizzle
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint32_t off = hc * (kPBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPh + off), "r"(ph[4 * c]),
-                             "r"(ph[4 * c + 1]), "r"(ph[4 * c + 2]), "r"(ph[4 * c + 3])
-                             : "memory");
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(sPl + off), "r"(pl[4 * c]),
-                             "r"(pl[4 * c + 1]), "r"(pl[4 * c + 2]), "r"(pl[4 * c + 3])
-                             : "memory");
-            }
-            l_half = l_half * alpha + sum;
-            m_used = m_new;
-            // keys past the end of the sequence: zero their V rows (P is 0 there, V may be stale)
-            if (t == ntiles - 1 && t * kBN + kBN > seq_len) {
+            // keys past the end of the sequence: zero their V rows (P is 0 there, V may be
+            // stale).  Tile A's warps do it before their P . V, which runs before tile B's.
+            if (x == 0 && t == ntiles - 1 && key0 + kBN > seq_len) {
                 const int s = t % kNS;
                 if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
                     ok = false;
                     break;
                 }
-                const int first = seq_len - t * kBN;
-                const int tid = threadIdx.x - 64;             // 0..255
-                for (int i = tid; i < 2 * (kBN - first) * 8; i += 256) {
+                const int first = seq_len - key0;
+                const int tid = threadIdx.x - 64;             // 0..127
+                for (int i = tid; i < 2 * (kBN - first) * 8; i += 128) {
                     const int x16 = i & 7, rowi = (i >> 3) % (kBN - first), half = (i >> 3) / (kBN - first);
                     const uint32_t a = sV + s * kKVBytes + half * (kKVBytes / 2) + (first + rowi) * 128 + x16 * 16;
                     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
+            if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[x]));
         }
-        float l_tot = l_half;
-        if (ok) l_tot += exchange(l_half, ntiles);
-        if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), (ntiles - 1) & 1, &s_abort, p.status))) {
+        if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done[x]), 0, &s_abort, p.status))) {
             tc_fence_after();
             const bool valid = pos < p.C;
-            const float inv = p.cascade ? 1.f : 1.f / l_tot;
+            const float inv = p.cascade ? 1.f : 1.f / l_run;
             const size_t qrow = (size_t)pos * p.H_q + g * p.G + (r % p.G);
-            float* orow = (p.cascade ? p.ws_o + qrow * p.slots * kD : p.out + qrow * kD) + (kD / 2) * hc;
-            if (p.cascade && valid && hc == 0)
-                *reinterpret_cast<float2*>(p.ws_ml + qrow * p.slots * 2) = make_float2(m_used, l_tot);
+            float* orow = p.cascade ? p.ws_o + qrow * p.slots * kD : p.out + qrow * kD;
+            if (p.cascade && valid)
+                *reinterpret_cast<float2*>(p.ws_ml + qrow * p.slots * 2) = make_float2(m_used, l_run);
 #pragma unroll 1
-            for (int c = 0; c < kD / 64; ++c) {
+            for (int c = 0; c < kD / 32; ++c) {
                 float o[32];
-                tmem_ld32(trow + 2 * kBN + (kD / 2) * hc + 32 * c, o);
+                tmem_ld32(tO + 32 * c, o);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
@@ -584,7 +577,7 @@ int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtens
     auto kern = a.kv_dtype == PKV_BF16 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
         return PKV_ERR_CUDA;
-    const int pos_per_cta = kBM / a.G;
+    const int pos_per_cta = kQT * (kBM / a.G);
     const dim3 grid((a.C + pos_per_cta - 1) / pos_per_cta, a.H_kv);
     kern<<<grid, kThreads, kSmem, s>>>(p, *tmq, *tmk, *tmv);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
