@@ -32,35 +32,43 @@ namespace pkv {
 // ---------------------------------------------------------------------------
 // Tensor-core engine, 16-bit pools.
 // ---------------------------------------------------------------------------
-template <int D, int STAGES>
+template <int D, int STAGES, int NW>
 struct Mma16Cfg {
     static constexpr int TILE = 16 * 2 * D;        // bytes of one K (or V) tile
     static constexpr int NBOX = D / 64;            // 128-byte boxes per row
     static constexpr int STAGE = 2 * TILE;
-    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static constexpr int RING = STAGES * STAGE;
+    static constexpr int STAGING = NW * 16 * (D + 4) * 4;   // the epilogue's 16 O rows per warp
+    static constexpr int BODY = RING > STAGING ? RING : STAGING;
+    static constexpr int SMEM = BODY + 1024;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
-    static_assert(STAGES * STAGE >= 16 * (D + 4) * 4, "the epilogue stages 16 O rows in the ring");
 };
 
-template <int D, bool BF16, int NHT, int STAGES>
-__global__ void __launch_bounds__(32)
+// NW = 1: one warp per (partition, KV head or group of 16 of its query heads, sequence).
+// NW > 1 (groups of 17..64 query heads): NW warps share one K/V ring, warp w taking query
+// heads 16w .. 16w+15 of the group, so every K/V tile crosses into the SM once; a stage is
+// refilled once all warps have released it.
+template <int D, bool BF16, int NHT, int STAGES, int NW>
+__global__ void __launch_bounds__(32 * NW)
 decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV)
 {
-    using Cfg = Mma16Cfg<D, STAGES>;
+    using Cfg = Mma16Cfg<D, STAGES, NW>;
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[STAGES];
+    __shared__ __align__(8) uint64_t empty[STAGES];
     __shared__ int tbl[kMaxPartTiles];
 
     pdl_launch_dependents();   // the split-K merge may be scheduled behind the last wave
-    const int lane = threadIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int part = blockIdx.x, b = blockIdx.z;
-    const int g = blockIdx.y / p.hgroups, hg = blockIdx.y - g * p.hgroups;   // KV head, group of 16 heads
-    const int GC = min(16, p.G - 16 * hg);                                   // query heads of this CTA
+    const int g = NW > 1 ? blockIdx.y : blockIdx.y / p.hgroups;               // KV head
+    const int hg = NW > 1 ? warp : blockIdx.y - g * p.hgroups;                // group of 16 query heads
+    const int GC = min(16, p.G - 16 * hg);                                   // query heads of this warp
     const int r = lane >> 2, qd = lane & 3;
     const int hbase = g * p.G + 16 * hg;
 
-    const int ctx = checked_ctx(p, b, lane == 0 && part == 0 && g == 0);
+    const int ctx = checked_ctx(p, b, threadIdx.x == 0 && part == 0 && g == 0);
     const int nparts = part_count(p, ctx);
     const int tok0 = seq_base(p, ctx) + part * p.part_tokens;
     const int lo = visible_lo(p, ctx);   // tokens before lo are outside the window
@@ -75,7 +83,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     const int ntiles = (ntok + kBlock - 1) / kBlock;
 
     const int32_t* trow = p.tables + (size_t)b * p.W + tok0 / kBlock;
-    for (int j = lane; j < ntiles; j += 32) {
+    for (int j = threadIdx.x; j < ntiles; j += 32 * NW) {
         int blk = trow[j];
         if ((unsigned)blk >= (unsigned)p.N) {
             flag_status(p.status, PKV_DEV_BAD_BLOCK);
@@ -84,13 +92,16 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         tbl[j] = blk;
     }
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    if (lane == 0) {
-        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);
+            mbar_init(smem_u32(&empty[s]), NW);
+        }
         mbar_fence_init();
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
     }
-    __syncwarp();
+    __syncthreads();
 
     auto issue = [&](int j) {
         const int s = j % STAGES;
@@ -103,7 +114,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 #pragma unroll
         for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + Cfg::TILE + x * 2048, &tmV, x * 64, row, bar);
     };
-    if (lane == 0) {
+    if (threadIdx.x == 0) {
         for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
     }
 
@@ -243,9 +254,25 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         }
 
         __syncwarp();
-        if (lane == 0 && j + STAGES < ntiles) {
-            fence_proxy_async_smem();
-            issue(j + STAGES);
+        if constexpr (NW == 1) {
+            if (lane == 0 && j + STAGES < ntiles) {
+                fence_proxy_async_smem();
+                issue(j + STAGES);
+            }
+        } else {   // release the stage; thread 0 refills it once every warp has
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                mbar_arrive(smem_u32(&empty[s]));
+            }
+            if (threadIdx.x == 0 && j + STAGES < ntiles) {
+                if (mbar_wait_bounded(smem_u32(&empty[s]), (j / STAGES) & 1)) {
+                    issue(j + STAGES);
+                } else {
+                    ok = false;
+                    ++j;
+                    break;
+                }
+            }
         }
     }
 
@@ -253,14 +280,15 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
         for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
             mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
-        return;
     }
+    if constexpr (NW > 1) __syncthreads();   // every warp is done with the ring before the staging reuses it
+    if (!ok) return;
 
     // ---- epilogue: O rows [head][dim] through shared memory, then coalesced stores
 #pragma unroll
     for (int hr = 0; hr < NHT; ++hr) l_run[hr] = warp_sum_quad(l_run[hr]);
     const bool final_out = (p.part_base == 0 && nparts == 1);
-    float* so = reinterpret_cast<float*>(smem);
+    float* so = reinterpret_cast<float*>(smem) + warp * 16 * (D + 4);
     constexpr int SR = D + 4;   // padded row stride (floats)
     __syncwarp();
 #pragma unroll
@@ -371,22 +399,38 @@ namespace {
 constexpr int kStages = 4;
 
 template <typename K>
-int launch_k(K kernel, int smem, dim3 grid, cudaStream_t s, const DecodeParams& p, const CUtensorMap* tmk,
-             const CUtensorMap* tmv)
+int launch_k(K kernel, int smem, dim3 grid, int threads, cudaStream_t s, const DecodeParams& p,
+             const CUtensorMap* tmk, const CUtensorMap* tmv)
 {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return PKV_ERR_CUDA;
-    kernel<<<grid, 32, smem, s>>>(p, *tmk, *tmv);
+    kernel<<<grid, threads, smem, s>>>(p, *tmk, *tmv);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
+template <int D, bool BF16, int NW>
+int launch_mma16_nw(const DecodeParams& p, int nht, dim3 grid, cudaStream_t s, const CUtensorMap* tmk,
+                    const CUtensorMap* tmv)
+{
+    constexpr int smem = Mma16Cfg<D, kStages, NW>::SMEM;
+    if (nht == 1)
+        return launch_k(decode_mma16_kernel<D, BF16, 1, kStages, NW>, smem, grid, 32 * NW, s, p, tmk, tmv);
+    return launch_k(decode_mma16_kernel<D, BF16, 2, kStages, NW>, smem, grid, 32 * NW, s, p, tmk, tmv);
+}
+
+// Groups of 17..64 query heads run as one CTA of ceil(G / 16) warps sharing the K/V ring;
+// wider groups as one single-warp CTA per 16 heads.
 template <int D, bool BF16>
 int launch_mma16(const DecodeParams& p, int nht, dim3 grid, cudaStream_t s, const CUtensorMap* tmk,
                  const CUtensorMap* tmv)
 {
-    constexpr int smem = Mma16Cfg<D, kStages>::SMEM;
-    if (nht == 1) return launch_k(decode_mma16_kernel<D, BF16, 1, kStages>, smem, grid, s, p, tmk, tmv);
-    return launch_k(decode_mma16_kernel<D, BF16, 2, kStages>, smem, grid, s, p, tmk, tmv);
+    const dim3 g1(grid.x, grid.y / p.hgroups, grid.z);   // one CTA per KV head
+    switch (p.hgroups) {
+    case 2: return launch_mma16_nw<D, BF16, 2>(p, nht, g1, s, tmk, tmv);
+    case 3: return launch_mma16_nw<D, BF16, 3>(p, nht, g1, s, tmk, tmv);
+    case 4: return launch_mma16_nw<D, BF16, 4>(p, nht, g1, s, tmk, tmv);
+    default: return launch_mma16_nw<D, BF16, 1>(p, nht, grid, s, tmk, tmv);
+    }
 }
 
 }  // namespace
