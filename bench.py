@@ -167,6 +167,10 @@ WORKLOADS = {
                    lens="long", pool_blocks=64 * 2048, window=4096,
                    desc="sliding-window decode, 1 layer of the 70B shape (H_q 64, H_kv 8, d 128, bf16), B 64, "
                         "ctx ~ U[16384, 32768], window 4,096 tokens: only the window's K/V is read"),
+    "blocks": dict(kind="blocks", layers=80, H_kv=8, d=128, dtype=wl.BF16, pool_blocks=4096, copies=512, swaps=16,
+                   desc="whole-block moves on the 80-layer 70B-class bf16 pool (a block = 80 layers x K and V of 8 "
+                        "heads, 5.24 MB): copy-on-write of 512 blocks, swap-out of 16 blocks to pinned host memory "
+                        "and swap-in of 16"),
     "prefix_chunk": dict(kind="prefix", layers=1, B=256, H_q=64, H_kv=8, d=128, dtype=wl.BF16,
                          desc="prefix sharing + chunked prefill, 1 layer of the 70B shape, bf16: 256 decodes "
                               "share a 4,000-token prefix (250 blocks) + private 200-token suffixes + U{0..300} "
@@ -453,6 +457,74 @@ def build_prefix_chunk(args, cfg, dev, rank):
     return step, e2e_step, info, pool
 
 
+def build_blocks(args, cfg, dev, rank):
+    """Whole-block moves on the 80-layer 70B-class pool: one step copies `copies` blocks
+    (copy-on-write at divergence) and swaps `swaps` blocks out to pinned host memory and
+    back in (preemption).  Block = all layers' K and V tiles of its 8 KV heads (5.24 MB)."""
+    from paged_kv_cache_431_b200 import pkv
+
+    L, H_kv, d, N = cfg["layers"], cfg["H_kv"], cfg["d"], cfg["pool_blocks"]
+    n_copy, n_swap = cfg["copies"], cfg["swaps"]
+    gd = wl.generator(431 + 500 + rank, dev)
+    k_pool = torch.empty(L, N, H_kv, 16, d, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.empty_like(k_pool)
+    for l in range(L):
+        k_pool[l] = wl.normal((N, H_kv, 16, d), torch.bfloat16, gd, dev)
+        v_pool[l] = wl.normal((N, H_kv, 16, d), torch.bfloat16, gd, dev)
+    pool = pkv.KVPool(k_pool, v_pool, wl.BF16, d, device_status=torch.zeros(1, dtype=torch.int32, device=dev))
+    gen = wl.generator(431 + 6 + rank)
+    perm = torch.randperm(N, generator=gen).to(torch.int32)
+    src = perm[:n_copy].contiguous()
+    dst = perm[n_copy:2 * n_copy].contiguous()
+    out_ids = perm[2 * n_copy:2 * n_copy + n_swap].contiguous()
+    in_ids = perm[2 * n_copy + n_swap:2 * n_copy + 2 * n_swap].contiguous()
+    d_src, d_dst, d_out, d_in = (t.to(dev) for t in (src, dst, out_ids, in_ids))
+    per_block = pkv.kv_swap_bytes_per_block(pool)
+    host = torch.empty(n_swap, per_block, dtype=torch.uint8).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0][0].record(stream)
+        pkv.kv_copy_blocks(pool, d_src, d_dst)
+        if ev is not None:
+            ev[0][1].record(stream)
+            ev[1][0].record(stream)
+        pkv.kv_swap_out(pool, d_out, host)
+        if ev is not None:
+            ev[1][1].record(stream)
+            ev[2][0].record(stream)
+        pkv.kv_swap_in(pool, d_in, host)
+        if ev is not None:
+            ev[2][1].record(stream)
+
+    # end to end: the block ids come from pinned host memory every step
+    h_ids = torch.cat([src, dst, out_ids, in_ids]).pin_memory()
+    d_ids = torch.empty_like(h_ids, device=dev)
+
+    def e2e_step():
+        d_ids.copy_(h_ids, non_blocking=True)
+        pkv.kv_copy_blocks(pool, d_ids[:n_copy], d_ids[n_copy:2 * n_copy])
+        pkv.kv_swap_out(pool, d_ids[2 * n_copy:2 * n_copy + n_swap], host)
+        pkv.kv_swap_in(pool, d_ids[2 * n_copy + n_swap:], host)
+
+    copied = n_copy * per_block
+    swapped = n_swap * per_block
+    peaks, kind = measured_peaks()
+    info = dict(
+        config={"workload": args.workload, "description": cfg["desc"], "layers": L, "kv_heads": H_kv, "head_dim": d,
+                "kv_dtype": "bf16", "pool_blocks_per_layer": N, "copy_pairs": n_copy, "swapped_blocks": n_swap,
+                "bytes_per_block": per_block, "parallelism": "replicas",
+                "l2": f"inputs larger than L2: each copy call moves {copied / 1e9:.2f} GB"},
+        kv_bytes_per_step=copied + 2 * swapped, seq_tokens_per_step=(n_copy + 2 * n_swap) * 16 * L, layers=L,
+        roofline=dict(bound="hbm", kernel="kv_copy_blocks", alg_bytes=2 * copied, call_index=0,
+                      peak=float(peaks["hbm_gbs"]), unit="GB/s",
+                      peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs; a copy reads and writes each byte)",
+                      traffic=None, swap_bytes=swapped),
+        launches_per_step=3, dtype="u8", h2d=h_ids.numel() * 4 + swapped, d2h=swapped, calls_per_step=3)
+    return step, e2e_step, info, pool
+
+
 def max_over_ranks(value: float, device) -> float:
     """The largest `value` over all ranks: the slowest replica bounds the whole job.  The
     identity without a process group (one GPU)."""
@@ -499,7 +571,7 @@ def run_gpu(args):
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
     cfg = WORKLOADS[args.workload]
-    builder = build_prefix_chunk if cfg["kind"] == "prefix" else build_decode
+    builder = {"prefix": build_prefix_chunk, "blocks": build_blocks}.get(cfg["kind"], build_decode)
     step, e2e_step, info, pool = builder(args, cfg, dev, rank)
 
     for _ in range(args.warmup):
@@ -528,12 +600,17 @@ def run_gpu(args):
     call_ms = timed.call_ms()
     rf = info["roofline"]
     if rf["bound"] == "hbm":
-        avg_s = statistics.mean(call_ms) * 1e-3
+        cpk = info["calls_per_step"]
+        sel = call_ms if "call_index" not in rf else call_ms[rf["call_index"]::cpk]
+        avg_s = statistics.mean(sel) * 1e-3
         achieved = rf["alg_bytes"] / avg_s / 1e9
         roofline = {"bound": "hbm", "kernel": rf["kernel"], "achieved": round(achieved, 1), "peak": rf["peak"],
                     "unit": "GB/s", "frac": round(achieved / rf["peak"], 4), "peak_source": rf["peak_source"],
                     "traffic": rf["traffic"], "algorithmic_bytes_per_launch": rf["alg_bytes"],
                     "avg_launch_us": round(avg_s * 1e6, 2)}
+        if "swap_bytes" in rf:   # host-link moves: swap-out then swap-in calls
+            for name, i in (("swap_out_gbs", 1), ("swap_in_gbs", 2)):
+                roofline[name] = round(rf["swap_bytes"] / (statistics.mean(call_ms[i::cpk]) * 1e-3) / 1e9, 2)
     else:
         ci = rf["call_index"]
         per_call = [call_ms[i] for i in range(ci, len(call_ms), info["calls_per_step"])]
@@ -582,6 +659,8 @@ def cpu_oracle(workload, budget_s=12.0, per_step=None, steps=None, warmup=0):
 
     oracle.build()
     cfg = WORKLOADS[workload]
+    if cfg["kind"] == "blocks":
+        return cpu_oracle_blocks(cfg, workload, budget_s, per_step, steps, warmup)
     H_q, H_kv, d, dt = cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
     gen = wl.generator(431 + 3)
     if cfg["kind"] == "prefix":
@@ -627,6 +706,42 @@ def cpu_oracle(workload, budget_s=12.0, per_step=None, steps=None, warmup=0):
     return (res, step_secs) if per_step else res
 
 
+def cpu_oracle_blocks(cfg, workload, budget_s, per_step=None, steps=None, warmup=0):
+    """The oracle's block copy (numpy byte moves, every layer) on a bounded sample of pairs
+    from a small pool of the same shape."""
+    import oracle
+
+    L, H_kv, d = cfg["layers"], cfg["H_kv"], cfg["d"]
+    n_blocks, pairs = 64, per_step or 16
+    rng = np.random.default_rng(431)
+    pools = []
+    for _ in range(L):
+        pl = oracle.Pool(n_blocks, H_kv, d, oracle.BF16)
+        pl.k[...] = rng.integers(0, 256, pl.k.shape, dtype=np.uint8)
+        pl.v[...] = rng.integers(0, 256, pl.v.shape, dtype=np.uint8)
+        pools.append(pl)
+    per_block = L * 2 * H_kv * 16 * d * 2
+    total_s, moved, step_secs, s = 0.0, 0, [], 0
+    n_steps = (warmup + steps) if per_step else 10 ** 9
+    while s < n_steps:
+        perm = rng.permutation(n_blocks)
+        t0 = time.perf_counter()
+        oracle.copy_blocks(pools, perm[:pairs], perm[pairs:2 * pairs])
+        dt = time.perf_counter() - t0
+        if s >= warmup:
+            total_s += dt
+            moved += pairs * per_block
+            step_secs.append(dt)
+        s += 1
+        if not per_step and total_s >= budget_s:
+            break
+    res = {"value": round(moved / total_s / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "seq_tokens_per_s_per_layer": round(moved / per_block * 16 / total_s),
+           "sample": f"{len(step_secs)} x {pairs} block copies of the {workload} shape ({L} layers, numpy), "
+                     f"single thread, {total_s:.1f} s"}
+    return (res, step_secs) if per_step else res
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle on this host, same workload, metric and unit;
     each step is a bounded sample (--ref-seqs whole sequences of one layer)."""
@@ -636,7 +751,9 @@ def run_reference(args):
     cpu, secs = cpu_oracle(args.workload, per_step=max(1, args.ref_seqs), steps=args.steps, warmup=args.warmup)
     res = {"metric": METRIC, "value": cpu["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 2), "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "scaling": "weak", "vs_baseline": None,
+           "dtype": "u8" if WORKLOADS[args.workload]["kind"] == "blocks" else "f64", "data": "synthetic",
+           "impl": "reference",
            "config": {"workload": args.workload, "description": WORKLOADS[args.workload]["desc"]},
            "seq_tokens_per_s_per_layer": cpu["seq_tokens_per_s_per_layer"],
            "cpu_baseline": cpu,

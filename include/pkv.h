@@ -218,9 +218,10 @@ PKV_API int paged_decode_attn_noalloc(pkv_pool_t pool, int layer, const void* q,
                                       int max_context_len, float scale, float* out,
                                       const pkv_decode_opts* opts, void* stream);
 
-/* Workspace paged_decode_attn_cascade needs (bytes): num_seqs * num_q_heads * (1 + suffix
- * partitions) * (head_dim + 2) * 4.  0 for an unsupported shape.  With shared_prefix_len 0
- * it equals paged_decode_workspace_bytes. */
+/* Workspace paged_decode_attn_cascade needs (bytes): num_seqs * num_q_heads * (prefix key
+ * splits + suffix partitions) * (head_dim + 2) * 4, the prefix split over as many CTAs as
+ * fill the GPU.  0 for an unsupported shape.  With shared_prefix_len 0 it equals
+ * paged_decode_workspace_bytes. */
 PKV_API size_t paged_decode_cascade_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads,
                                                     int max_context_len, int shared_prefix_len,
                                                     const pkv_decode_opts* opts);

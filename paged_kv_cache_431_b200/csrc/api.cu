@@ -350,7 +350,9 @@ size_t paged_decode_cascade_workspace_bytes(pkv_pool_t pool, int num_seqs, int n
     if (cascade_partitioning(pool, num_seqs, num_q_heads, max_context_len, shared_prefix_len, opts, &P, &parts) !=
         PKV_OK)
         return 0;
-    return (size_t)num_seqs * num_q_heads * (1 + parts) * (pool->d.head_dim + 2) * sizeof(float);
+    const int splits = prefill_tc_key_splits(num_seqs, num_q_heads / pool->d.num_kv_heads, pool->d.num_kv_heads,
+                                             shared_prefix_len);
+    return (size_t)num_seqs * num_q_heads * (splits + parts) * (pool->d.head_dim + 2) * sizeof(float);
 }
 
 int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_dtype, const int32_t* block_tables,
@@ -383,7 +385,9 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     int P, parts;
     int rc = cascade_partitioning(pool, num_seqs, num_q_heads, max_context_len, shared_prefix_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;
-    const int slots = 1 + parts;
+    const int G = num_q_heads / d.num_kv_heads;
+    const int splits = prefill_tc_key_splits(num_seqs, G, d.num_kv_heads, shared_prefix_len);
+    const int slots = splits + parts;   // prefix partials in slots 0 .. splits-1, then the suffix
     const size_t need = (size_t)num_seqs * num_q_heads * slots * (d.head_dim + 2) * sizeof(float);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15)) return PKV_ERR_WORKSPACE;
     const CUtensorMap *tmk = nullptr, *tmv = nullptr;
@@ -391,7 +395,6 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     if (rc != PKV_OK) return rc;
     float* ws_o = static_cast<float*>(workspace);
     float* ws_ml = ws_o + (size_t)num_seqs * num_q_heads * slots * d.head_dim;
-    const int G = num_q_heads / d.num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     // 1. the shared prefix, once per KV group for the whole batch, on the tensor cores:
@@ -413,6 +416,7 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     pa.out = nullptr;
     pa.status = d.device_status;
     pa.cascade_nkeys = shared_prefix_len;
+    pa.key_splits = splits;
     pa.ws_slots = slots;
     pa.ws_o = ws_o;
     pa.ws_ml = ws_ml;
@@ -447,7 +451,7 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     a.status = d.device_status;
     a.engine = engine;
     a.tok_base = shared_prefix_len;
-    a.part_base = 1;
+    a.part_base = splits;
     return launch_decode(a, tmk, tmv, s);
 }
 

@@ -339,8 +339,8 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 // ---------------------------------------------------------------------------
 // Split-K merge: out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
 // One warp per (query head, sequence); sequences that fit one partition were written
-// directly by the main kernel and are skipped.  In the shared-prefix (cascade) form slot 0
-// holds the prefix's partial and the suffix partitions follow.
+// directly by the main kernel and are skipped.  In the shared-prefix (cascade) form slots
+// 0 .. part_base-1 hold the prefix's partials (one per key split) and the suffix follows.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)

@@ -22,7 +22,8 @@ struct DecodeParams {
     int W, H_q, H_kv, G, N, part_tokens, max_parts;
     // Partitions cover tokens tok_base .. ctx-1 and write workspace slots part_base + part of
     // a row of `slots`.  Plain decode: 0, 0, max_parts.  Shared-prefix (cascade) decode:
-    // tok_base = prefix length, part_base = 1 (slot 0 holds the prefix's partial).
+    // tok_base = prefix length, part_base = key splits of the prefix (slots 0 .. part_base-1
+    // hold the prefix's partials).
     int tok_base, part_base, slots;
     int prefix_blocks;      // cascade: table entries every sequence must share with row 0
     int window;             // sliding window: tokens a query sees (0: the whole context)

@@ -82,9 +82,11 @@ struct PrefillArgs {
     int32_t* status;
     // tcgen05 form only: shared-prefix (cascade) pass of the decode.  With cascade_nkeys > 0
     // the C positions are the decode batch, every row sees keys 0 .. cascade_nkeys-1, and the
-    // partial (o, m, l) goes to slot 0 of decode workspace rows of ws_slots slots.
+    // partials (o, m, l) of the key_splits key ranges go to slots 0 .. key_splits-1 of decode
+    // workspace rows of ws_slots slots.
     int window = 0;         // sliding window (warp-level form only)
     int cascade_nkeys = 0;
+    int key_splits = 1;     // cascade: CTAs the prefix keys are split over (partials in slots 0..)
     int ws_slots = 0;
     float* ws_o = nullptr;
     float* ws_ml = nullptr;
@@ -97,6 +99,8 @@ PFN_encode tensor_map_encoder();   // null when no driver is present
 
 // tcgen05 / TMEM form of the chunked prefill (prefill_tc.cu)
 bool prefill_tc_supported(int d, int G, int kv_dtype);
+// Key splits of the cascade prefix pass that fill the GPU (>= 1, <= key tiles).
+int prefill_tc_key_splits(int C, int G, int H_kv, int nkeys);
 bool make_q_map(CUtensorMap* map, const void* q, int C, int H_q, int G, PFN_encode enc);
 int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtensorMap* tmk, const CUtensorMap* tmv,
                       cudaStream_t s);

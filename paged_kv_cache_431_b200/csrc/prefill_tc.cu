@@ -53,7 +53,9 @@ struct TcParams {
     float scale_log2;
     // Shared-prefix (cascade) form: the C "positions" are C sequences whose query rows all
     // see the same nkeys keys (no causal mask); the unnormalized output and (m, l) go to
-    // slot 0 of the decode workspace rows [C][H_q][slots] instead of `out`.
+    // the decode workspace rows [C][H_q][slots] instead of `out`.
+    // The cascade form may split the keys over gridDim.z CTAs per query tile pair, split z
+    // writing slot z (a small batch alone would leave most SMs idle).
     int cascade, nkeys, slots;
     float* ws_o;
     float* ws_ml;
@@ -207,7 +209,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
     const int i_end = min(p.C, i0 + kQT * pos_per_tile);
     const int seq_len = p.cascade ? p.nkeys : p.P0 + p.C;
     const int kend = p.cascade ? p.nkeys : p.P0 + i_end;     // exclusive key bound of the CTA's last row
-    const int ntiles = (kend + kBN - 1) / kBN;
+    const int ntiles_all = (kend + kBN - 1) / kBN;
+    const int t_lo = (int)((long)blockIdx.z * ntiles_all / gridDim.z);        // this CTA's key tiles
+    const int t_hi = (int)((long)(blockIdx.z + 1) * ntiles_all / gridDim.z);
+    const int ntiles = t_hi - t_lo;                          // tile t_lo + u is the u-th of this CTA
     const int nblk_seq = (seq_len + kBlock - 1) / kBlock;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -269,14 +274,15 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 tma_load_3d(sQ + x * kQBytes + kQBytes / 2, &tmQ, 64, g * p.G, i0 + x * pos_per_tile, qb);
             }
         }
-        int cur = table_entry(lane);                         // chunk 0
-        int nxt = table_entry(32 + lane);                    // chunk 1
+        const int lb0 = t_lo * kBlkPerTile;                  // first logical block of this CTA
+        int cur = table_entry(lb0 + lane);                   // chunk 0
+        int nxt = table_entry(lb0 + 32 + lane);              // chunk 1
         int issued = 0, issued_k = 0;                        // tiles whose V (K) copies were issued
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = 0; t < ntiles; ++t) {                   // t counts this CTA's tiles
             const int s = t % kNS;
             if (t > 0 && t % kTilesPerChunk == 0) {
                 cur = nxt;
-                nxt = table_entry((t / kTilesPerChunk + 1) * 32 + lane);
+                nxt = table_entry(lb0 + (t / kTilesPerChunk + 1) * 32 + lane);
             }
             int row_of[kBlkPerTile];
 #pragma unroll
@@ -412,7 +418,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             }
             tc_fence_after();
             // pass 1: the row maximum over the tile's 128 scores (64 at a time)
-            const int key0 = t * kBN;
+            const int key0 = (t_lo + t) * kBN;
             const bool need_mask = key0 + kBN > kmin_tile;
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
@@ -485,7 +491,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             }
             // keys past the end of the sequence: zero their V rows (P is 0 there, V may be
             // stale).  Tile A's warps do it before their P . V, which runs before tile B's.
-            if (x == 0 && t == ntiles - 1 && key0 + kBN > seq_len) {
+            if (x == 0 && t == ntiles - 1 && key0 + kBN > seq_len) {   // only the last split's last tile
                 const int s = t % kNS;
                 if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
                     ok = false;
@@ -510,9 +516,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             const bool valid = pos < p.C;
             const float inv = p.cascade ? 1.f : 1.f / l_run;
             const size_t qrow = (size_t)pos * p.H_q + g * p.G + (r % p.G);
-            float* orow = p.cascade ? p.ws_o + qrow * p.slots * kD : p.out + qrow * kD;
+            const size_t slot = qrow * p.slots + blockIdx.z;
+            float* orow = p.cascade ? p.ws_o + slot * kD : p.out + qrow * kD;
             if (p.cascade && valid)
-                *reinterpret_cast<float2*>(p.ws_ml + qrow * p.slots * 2) = make_float2(m_used, l_run);
+                *reinterpret_cast<float2*>(p.ws_ml + slot * 2) = make_float2(m_used, l_run);
 #pragma unroll 1
             for (int c = 0; c < kD / 32; ++c) {
                 float o[32];
@@ -537,6 +544,15 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
 }
 
 }  // namespace
+
+int prefill_tc_key_splits(int C, int G, int H_kv, int nkeys)
+{
+    const int ctas = (C + kQT * (kBM / G) - 1) / (kQT * (kBM / G)) * H_kv;
+    const int tiles = (nkeys + kBN - 1) / kBN;
+    int z = num_sms() / (ctas > 0 ? ctas : 1);
+    z = z < 1 ? 1 : z;
+    return z < tiles ? z : tiles;
+}
 
 bool prefill_tc_supported(int d, int G, int kv_dtype)
 {
@@ -578,7 +594,7 @@ int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtens
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
         return PKV_ERR_CUDA;
     const int pos_per_cta = kQT * (kBM / a.G);
-    const dim3 grid((a.C + pos_per_cta - 1) / pos_per_cta, a.H_kv);
+    const dim3 grid((a.C + pos_per_cta - 1) / pos_per_cta, a.H_kv, a.cascade_nkeys > 0 ? a.key_splits : 1);
     kern<<<grid, kThreads, kSmem, s>>>(p, *tmq, *tmk, *tmv);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
