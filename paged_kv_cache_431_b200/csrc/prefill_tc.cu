@@ -181,6 +181,28 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     return false;
 }
 
+// Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction.
+__device__ __forceinline__ unsigned long long f2bits(float2 a) { return *reinterpret_cast<unsigned long long*>(&a); }
+__device__ __forceinline__ float2 bitsf2(unsigned long long d) { return *reinterpret_cast<float2*>(&d); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)), "l"(f2bits(c)));
+    return bitsf2(d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
+{
+    unsigned long long d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)));
+    return bitsf2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)));
+    return bitsf2(d);
+}
+
 struct Bars {
     uint64_t q_full;
     uint64_t k_full[kNS];
@@ -444,7 +466,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             // the truncated remainder, both by byte permutes.
             // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
-            float sum = 0.f;
+            const float2 slx2 = make_float2(slx, slx), mref2 = make_float2(-mref, -mref);
+            float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 float v[32];
@@ -458,24 +481,24 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 uint32_t w[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(v[2 * e], slx, -mref));
-                    const float p1 = ex2(fmaf(v[2 * e + 1], slx, -mref));
+                    const float2 a = ffma2(make_float2(v[2 * e], v[2 * e + 1]), slx2, mref2);
+                    const float2 pp = make_float2(ex2(a.x), ex2(a.y));
                     if constexpr (BF16) {
-                        const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+                        const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
                         w[e] = __byte_perm(u0, u1, 0x7632);
-                        const float r0 = p0 - __uint_as_float(u0 & 0xffff0000u);
-                        const float r1 = p1 - __uint_as_float(u1 & 0xffff0000u);
-                        w[16 + e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                        const float2 rr = fsub2(pp, make_float2(__uint_as_float(u0 & 0xffff0000u),
+                                                                __uint_as_float(u1 & 0xffff0000u)));
+                        w[16 + e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                     } else {
-                        w[e] = pack2<false>(p0, p1);
+                        w[e] = pack2<false>(pp.x, pp.y);
                         const float2 back = unpack2<false>(w[e]);
-                        w[16 + e] = pack2<false>(p0 - back.x, p1 - back.y);
+                        w[16 + e] = pack2<false>(pp.x - back.x, pp.y - back.y);
                     }
-                    sum += p0 + p1;
+                    sum2 = fadd2(sum2, pp);
                 }
                 tmem_st32u(tS + 32 * c, w);
             }
-            l_run = l_run * alpha + sum;
+            l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;
             // the running max moved: rescale this row of O (P . V(t-1) is done: s_full(t) says so)
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
