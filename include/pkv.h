@@ -67,7 +67,7 @@ extern "C" {
 #define PKV_ERR_CUDA        -6   /* a CUDA runtime/driver call failed              */
 #define PKV_ERR_TIMEOUT     -7   /* a kernel gave up waiting on a copy (bounded)   */
 #define PKV_ERR_INDEX       -8   /* the device saw a bad block id / slot / length  */
-#define PKV_ERR_UNSUPPORTED -9   /* a supported-but-not-built configuration        */
+#define PKV_ERR_UNSUPPORTED -9   /* a shape or option the kernels do not handle      */
 
 /* device status bits (OR-ed into pkv_pool_desc.device_status) */
 #define PKV_DEV_BAD_BLOCK   0x1  /* block table entry outside [0, num_blocks)           */

@@ -131,7 +131,7 @@ const char* pkv_strerror(int status)
     case PKV_ERR_CUDA: return "a CUDA call failed";
     case PKV_ERR_TIMEOUT: return "a kernel gave up waiting on a bulk copy";
     case PKV_ERR_INDEX: return "the device saw a block id, slot or context length out of range";
-    case PKV_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case PKV_ERR_UNSUPPORTED: return "configuration not supported by the library";
     case PKV_ERR_NO_BLOCKS: return "not enough free blocks in the pool";
     case PKV_ERR_STATE: return "unknown, existing or swapped-out sequence, or a broken block-manager invariant";
     default: return "unknown status";

@@ -89,6 +89,14 @@ def lib() -> ctypes.CDLL:
     L.kv_swap_out.argtypes = [P, P, i32, P, P]
     L.kv_swap_in.restype = i32
     L.kv_swap_in.argtypes = [P, P, i32, P, P]
+    L.paged_decode_attn_noalloc.restype = i32
+    L.paged_decode_attn_noalloc.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, f32, P, P, P]
+    L.paged_decode_cascade_workspace_bytes.restype = sz
+    L.paged_decode_cascade_workspace_bytes.argtypes = [P, i32, i32, i32, i32, P]
+    L.paged_decode_attn_cascade.restype = i32
+    L.paged_decode_attn_cascade.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, i32, f32, P, P, sz, P, P]
+    L.paged_prefill_chunk_attn_window.restype = i32
+    L.paged_prefill_chunk_attn_window.argtypes = [P, i32, P, i32, P, i32, i32, i32, i32, f32, i32, P, P]
     L.pkv_read_device_status.restype = i32
     L.pkv_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
     _lib = L
@@ -247,12 +255,8 @@ def paged_decode_attn(pool: KVPool, layer: int, q: torch.Tensor, block_tables: t
 
 def paged_decode_cascade_workspace_bytes(pool: KVPool, num_seqs: int, num_q_heads: int, max_context_len: int,
                                         shared_prefix_len: int, engine: int = 0, partition_tokens: int = 0) -> int:
-    L = lib()
-    fn = L.paged_decode_cascade_workspace_bytes
-    fn.restype = ctypes.c_size_t
-    fn.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
-    return int(fn(pool.handle, num_seqs, num_q_heads, max_context_len, shared_prefix_len,
-                  _opts(engine, partition_tokens)))
+    return int(lib().paged_decode_cascade_workspace_bytes(pool.handle, num_seqs, num_q_heads, max_context_len,
+                                                          shared_prefix_len, _opts(engine, partition_tokens)))
 
 
 def paged_decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, block_tables: torch.Tensor,
@@ -262,11 +266,7 @@ def paged_decode_attn_cascade(pool: KVPool, layer: int, q: torch.Tensor, block_t
                               sliding_window: int = 0, stream=None) -> torch.Tensor:
     """Decode attention for a batch whose tables all start with the same shared_prefix_len
     tokens (row 0's blocks): the prefix is attended once per KV group on the tensor cores."""
-    L = lib()
-    fn = L.paged_decode_attn_cascade
-    P, i32 = ctypes.c_void_p, ctypes.c_int
-    fn.restype = i32
-    fn.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, i32, ctypes.c_float, P, P, ctypes.c_size_t, P, P]
+    fn = lib().paged_decode_attn_cascade
     B, H_q, d = q.shape
     if out is None:
         out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
@@ -293,11 +293,7 @@ def paged_decode_attn_noalloc(pool: KVPool, layer: int, q: torch.Tensor, block_t
     memory for one: the split-K partials use the library's fixed 32 MiB device buffer.  Only
     the output is the caller's.  Calls that may overlap on the GPU share that buffer and race;
     issue them in order on one stream."""
-    L = lib()
-    fn = L.paged_decode_attn_noalloc
-    P, i32 = ctypes.c_void_p, ctypes.c_int
-    fn.restype = i32
-    fn.argtypes = [P, i32, P, i32, P, i32, P, i32, i32, i32, ctypes.c_float, P, P, P]
+    fn = lib().paged_decode_attn_noalloc
     B, H_q, d = q.shape
     if out is None:
         out = torch.empty(B, H_q, d, dtype=torch.float32, device=q.device)
@@ -320,11 +316,7 @@ def paged_prefill_chunk_attn(pool: KVPool, layer: int, q: torch.Tensor, block_ta
                                               block_table.shape[-1], ctx_before, C, H_q, float(scale), _ptr(out),
                                               None, 0, _stream(stream)), "paged_prefill_chunk_attn")
         return out
-    L = lib()
-    fn = L.paged_prefill_chunk_attn_window
-    P, i32 = ctypes.c_void_p, ctypes.c_int
-    fn.restype = i32
-    fn.argtypes = [P, i32, P, i32, P, i32, i32, i32, i32, ctypes.c_float, i32, P, P]
+    fn = lib().paged_prefill_chunk_attn_window
     _check(fn(pool.handle, layer, _ptr(q), _dtype_code(q), _ptr(block_table), block_table.shape[-1], ctx_before, C,
               H_q, float(scale), int(sliding_window), _ptr(out), _stream(stream)), "paged_prefill_chunk_attn_window")
     return out
