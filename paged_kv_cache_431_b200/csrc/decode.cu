@@ -3,15 +3,19 @@
 // What is computed ("KV cache, continuous batching and paged attention", section "Paged
 // attention": the attention kernel follows the block table; "KV cache, GQA, paging and
 // continuous batching", section "Mechanics": G query heads share one KV head):
-//   out[b][h] = softmax_t(scale * q[b][h] . K_b[t]) V_b[t],  t < context_lens[b],
-// K_b[t] = tile (block_tables[b][t / 16], h / G), row t % 16.
+//   out[b][h] = softmax_t(scale * q[b][h] . K_b[t]) V_b[t],  lo_b <= t < context_lens[b],
+// K_b[t] = tile (block_tables[b][t / 16], h / G), row t % 16; lo_b = 0, or ctx - window with a
+// sliding window ("KV cache, continuous batching and paged attention", section "The KV
+// cache": sliding-window attention layers).
 //
 // Design (B200):
-//   * One warp per (partition of <= part_tokens tokens, KV head, sequence).  The warp
-//     streams its partition's (block, KV head) tiles -- 16 rows of K and of V, each tile
-//     contiguous in HBM -- into a ring of shared-memory stages with tiled TMA loads
-//     (128-byte swizzle, completion on an mbarrier; no multicast).  Lane 0 keeps STAGES
-//     tiles in flight; the block-table slice is read once into shared memory.
+//   * One warp per (partition of <= part_tokens tokens, KV head, sequence) and group of up
+//     to 16 query heads (wider groups: one CTA of ceil(G/16) warps sharing the K/V ring up
+//     to G = 64).  The CTA streams its partition's (block, KV head) tiles -- 16 rows of K
+//     and of V, each tile contiguous in HBM -- into a ring of shared-memory stages with
+//     tiled TMA loads (128-byte swizzle, completion on an mbarrier; no multicast).  One
+//     thread keeps STAGES tiles in flight; the block-table slice is read once into shared
+//     memory.
 //   * All G query heads of the KV group are processed together, so each K/V byte is
 //     read from HBM exactly once.  Q.K^T and P.V are small dense contractions
 //     (G x d times d x 16 tokens); they run on the tensor cores with warp-level
@@ -24,7 +28,9 @@
 //     shuffles.  Masked (past-the-end) tokens get -inf scores and zeroed V, so stale or
 //     poisoned slots never reach the result.
 //   * Split-K: a sequence longer than one partition writes per-partition (o, m, l)
-//     partials; decode_reduce merges them with the log-sum-exp rule.
+//     partials; decode_reduce merges them with the log-sum-exp rule.  The shared-prefix
+//     (cascade) form starts the partitions after the prefix and merges them with the
+//     prefix's partials written by the tensor-core prefill kernel.
 #include "decode_common.cuh"
 
 namespace pkv {

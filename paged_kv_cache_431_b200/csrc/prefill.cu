@@ -12,7 +12,10 @@
 // owns 16 query rows (row = position * G + head of one KV group), a CTA of 4 warps
 // shares K/V tiles of 64 keys (4 paged blocks, TMA-loaded with the 128-byte swizzle,
 // double-buffered), S = Q.K^T and O += P.V use mma.sync m16n8k16 with fp32
-// accumulation, and the online softmax keeps per-row running max / sum.
+// accumulation, and the online softmax keeps per-row running max / sum.  It serves the
+// shapes the tcgen05 form (prefill_tc.cu) does not: head dim 64, group sizes that do not
+// divide 128, and sliding-window chunks (a row at position p sees p - window + 1 .. p;
+// key tiles and blocks before every window of the CTA are not read).
 #include "common.cuh"
 #include "internal.h"
 
