@@ -48,6 +48,7 @@ PROFILES = os.path.join(ROOT, "profiles")
 DECODE_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_quant.cu",
                "paged_kv_cache_431_b200/csrc/decode_common.cuh", "paged_kv_cache_431_b200/csrc/common.cuh"]
 PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
+BLOCKS_SRCS = ["paged_kv_cache_431_b200/csrc/blocks.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
 
 
 # ------------------------------------------------------------------ utils --
@@ -521,7 +522,7 @@ def build_blocks(args, cfg, dev, rank):
         roofline=dict(bound="hbm", kernel="kv_copy_blocks", alg_bytes=2 * copied, call_index=0,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs; a copy reads and writes each byte)",
-                      traffic=None, swap_bytes=swapped),
+                      traffic=kernel_traffic("copy_blocks", BLOCKS_SRCS), swap_bytes=swapped),
         launches_per_step=3, dtype="u8", h2d=h_ids.numel() * 4 + swapped, d2h=swapped, calls_per_step=3)
     return step, e2e_step, info, pool
 
