@@ -31,31 +31,45 @@ __host__ __device__ inline size_t swap_block_bytes(const BlockGeom& g)
     return (size_t)g.L * 2 * g.tile_row + (size_t)g.L * 2 * g.scales * sizeof(float);
 }
 
-// One thread per 16 bytes of (pair, layer, K/V); scales by the first threads of each block.
-__global__ void copy_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g,
-                                   const int32_t* __restrict__ src, const int32_t* __restrict__ dst, int n,
-                                   int32_t* status)
+// One CTA per (pair, layer, K/V): the block's contiguous H_kv * 16 * row_bytes bytes of
+// that layer's K or V, copied with 16-byte vectors, each thread keeping kUnroll loads in
+// flight before its stores; the first threads also copy the scales.
+constexpr int kCopyThreads = 256;
+constexpr int kUnroll = 4;
+
+__global__ void __launch_bounds__(kCopyThreads)
+copy_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g, const int32_t* __restrict__ src,
+                   const int32_t* __restrict__ dst, int32_t* status)
 {
-    const size_t chunks = g.tile_row / 16;
-    const size_t per_pair = (size_t)g.L * 2 * chunks;
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= per_pair * n) return;
-    const int pr = (int)(i / per_pair);
-    size_t rem = i % per_pair;
-    const int layer = (int)(rem / (2 * chunks));
-    rem %= 2 * chunks;
-    const bool is_v = rem >= chunks;
-    const size_t c = rem % chunks;
+    const int item = blockIdx.x;                 // (pair * L + layer) * 2 + is_v
+    const bool is_v = item & 1;
+    const int layer = (item >> 1) % g.L;
+    const int pr = (item >> 1) / g.L;
     const int sb = src[pr], db = dst[pr];
     if ((unsigned)sb >= (unsigned)g.N || (unsigned)db >= (unsigned)g.N) {
-        if (c == 0 && layer == 0 && !is_v) flag_status(status, PKV_DEV_BAD_BLOCK);
+        if (threadIdx.x == 0 && layer == 0 && !is_v) flag_status(status, PKV_DEV_BAD_BLOCK);
         return;
     }
     uint8_t* base = (is_v ? v : k) + (size_t)layer * g.layer_bytes;
-    reinterpret_cast<uint4*>(base + (size_t)db * g.tile_row)[c] = reinterpret_cast<const uint4*>(base + (size_t)sb * g.tile_row)[c];
-    if (g.scales && c < g.scales) {
+    const uint4* from = reinterpret_cast<const uint4*>(base + (size_t)sb * g.tile_row);
+    uint4* to = reinterpret_cast<uint4*>(base + (size_t)db * g.tile_row);
+    const int chunks = (int)(g.tile_row / 16);
+    for (int c0 = threadIdx.x; c0 < chunks; c0 += kCopyThreads * kUnroll) {
+        uint4 t[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int c = c0 + u * kCopyThreads;
+            if (c < chunks) t[u] = from[c];
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int c = c0 + u * kCopyThreads;
+            if (c < chunks) to[c] = t[u];
+        }
+    }
+    if (g.scales) {
         float* sc = (is_v ? vs : ks) + (size_t)layer * g.layer_scales;
-        sc[(size_t)db * g.scales + c] = sc[(size_t)sb * g.scales + c];
+        for (size_t h = threadIdx.x; h < g.scales; h += kCopyThreads) sc[(size_t)db * g.scales + h] = sc[(size_t)sb * g.scales + h];
     }
 }
 
@@ -114,10 +128,12 @@ static int launch_moves(bool copy, const pkv_pool* pool, const int32_t* a, const
     if (grid > 0x7fffffffULL) return PKV_ERR_ARG;
     uint8_t* k = static_cast<uint8_t*>(pool->d.k_data);
     uint8_t* v = static_cast<uint8_t*>(pool->d.v_data);
-    if (copy)
-        copy_blocks_kernel<<<(unsigned)grid, threads, 0, s>>>(k, v, pool->d.k_scale, pool->d.v_scale, g, a, b, n,
-                                                              pool->d.device_status);
-    else
+    if (copy) {
+        const size_t items = (size_t)n * g.L * 2;
+        if (items > 0x7fffffffULL) return PKV_ERR_ARG;
+        copy_blocks_kernel<<<(unsigned)items, kCopyThreads, 0, s>>>(k, v, pool->d.k_scale, pool->d.v_scale, g, a, b,
+                                                                    pool->d.device_status);
+    } else
         swap_blocks_kernel<<<(unsigned)grid, threads, 0, s>>>(k, v, pool->d.k_scale, pool->d.v_scale, g, a, n, host,
                                                               to_host, pool->d.device_status);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
