@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kStages = 2;
 
 template <typename K>
 int launch_k(K kernel, int smem, dim3 grid, int threads, cudaStream_t s, const DecodeParams& p,
