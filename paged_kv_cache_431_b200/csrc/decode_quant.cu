@@ -32,7 +32,7 @@ struct QCfg {
     static constexpr int ROW = DT == PKV_INT4 ? D / 2 : D;     // bytes per token row
     static constexpr int TILE = 16 * ROW;                      // one (block, head) tile
     static constexpr int STAGE = 2 * TILE;                     // K and V
-    static constexpr int STAGES = DT == PKV_INT4 ? 4 : 3;
+    static constexpr int STAGES = DT == PKV_INT4 ? 3 : 2;
     static constexpr int RING = STAGES * STAGE;
     static constexpr int STAGING = 16 * (D + 4) * 4;           // epilogue: 16 O rows, fp32
     static constexpr int BODY = RING > STAGING ? RING : STAGING;   // the epilogue reuses the ring
