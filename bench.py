@@ -581,14 +581,28 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     if pkv.read_device_status(pool):
         raise RuntimeError("device status set during warm-up")
+    graph = None
+    if args.graph:   # the whole step (every layer's append and attention) as one CUDA graph
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(dev)
 
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    elapsed_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world)
+    # per-call durations (the roofline) from eager steps with events around each call
+    eager_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world)
+    elapsed_ms = eager_ms
+    if graph is not None:
+        elapsed_ms, _ = time_steps(lambda ev=None: graph.replay(), args.steps, 1, dev, world)
     clk = clocks.stop()
     if pkv.read_device_status(pool):
         raise RuntimeError("device status set during timing")
+    info["config"]["step_timing"] = ("CUDA-graph replays of one captured step" if graph is not None
+                                     else "eager launches") + f"; eager steps {eager_ms / args.steps:.4f} ms"
 
     # end to end through the same calls with host buffers
     for _ in range(max(1, args.warmup)):
@@ -779,6 +793,8 @@ def main():
                     help="split-K partition size in tokens (0: chosen by the library)")
     ap.add_argument("--decode-form", default="cascade", choices=["cascade", "plain"],
                     help="prefix_chunk: decode the shared-prefix batch in the cascade form or plainly")
+    ap.add_argument("--graph", type=int, default=1, choices=[0, 1],
+                    help="1: time the device-resident steps as replays of one CUDA-graph-captured step")
     ap.add_argument("--engine", type=int, default=0, choices=[0, 1, 2, 3],
                     help="decode engine: 0/1 tensor cores, 2 CUDA-core packed FMA, 3 CUDA-core FMA")
     args = ap.parse_args()
