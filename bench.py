@@ -45,8 +45,11 @@ from paged_kv_cache_431_b200 import workloads as wl  # noqa: E402
 
 METRIC = "paged GQA decode: KV HBM GB/s (% of ~8 TB/s peak); seq-tokens/s per layer"
 PROFILES = os.path.join(ROOT, "profiles")
-DECODE_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_quant.cu",
-               "paged_kv_cache_431_b200/csrc/decode_common.cuh", "paged_kv_cache_431_b200/csrc/common.cuh"]
+# the sources each kernel's DRAM-byte capture depends on (kernel, shared device code, launch setup)
+DECODE16_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
+                 "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
+DECODEQ_SRCS = ["paged_kv_cache_431_b200/csrc/decode_quant.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
+                "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
 BLOCKS_SRCS = ["paged_kv_cache_431_b200/csrc/blocks.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
 
@@ -347,7 +350,7 @@ def build_decode(args, cfg, dev, rank):
         roofline=dict(bound="hbm", kernel="paged_decode_attn (main + split-K merge)", alg_bytes=alg,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
-                      traffic=kernel_traffic(f"decode_{args.workload}", DECODE_SRCS)),
+                      traffic=kernel_traffic(f"decode_{args.workload}", DECODEQ_SRCS if quant else DECODE16_SRCS)),
         launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",
         h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L)
     return step, e2e_step, info, pool

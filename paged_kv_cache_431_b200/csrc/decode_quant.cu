@@ -8,11 +8,17 @@
 // Same structure as the 16-bit kernel (one warp per partition x KV head x sequence,
 // TMA ring of K/V code tiles, online softmax, split-K partials), with dequantization
 // fused into the fragment loads:
-//   * codes are converted to fp16 in registers -- int8 and int4 by the exponent
-//     trick (the code + bias placed in the mantissa of 1024.0, then the bias
-//     subtracted: exact), fp8 e4m3 by the hardware e4m3x2 -> f16x2 conversion
-//     (exact) -- and fed to mma.sync m16n8k16 (f16 in, fp32 accumulate); q is
-//     converted to fp16 once per warp;
+//   * codes are converted to fp16 in registers and fed to mma.sync m16n8k16 (f16 in,
+//     fp32 accumulate); q is converted to fp16 once per warp:
+//       - integer K codes: the code plus its offset (c + 128, c + 8) is moved into the
+//         significand of an fp16 subnormal (one byte permute or one logic op per pair,
+//         exact); the offset's share of every score, offset * sum(q), is subtracted once
+//         per score, and q is pre-scaled by a power of two so that its products with the
+//         subnormals stay well inside the accumulator's range;
+//       - integer V codes: the exponent trick (code + offset placed in the significand of
+//         1024.0, then 1024 + offset subtracted: exact) -- V meets the two-part P, whose
+//         low part times a subnormal loses precision in the tensor cores;
+//       - fp8 e4m3: the hardware e4m3x2 -> f16x2 conversion (exact);
 //   * the K scale of a tile multiplies that tile's scores, the V scale multiplies P
 //     before P . V, so the MMAs see plain integer-valued or fp8-valued operands;
 //   * which physical head dims feed which MMA k-slot is chosen so that every lane
@@ -89,33 +95,73 @@ __device__ __forceinline__ void load_run(uint32_t (&w)[BYTES / 4], uint32_t tile
     }
 }
 
+// K codes become fp16 SUBNORMALS: a half whose exponent field is 0 and whose significand
+// field holds the integer u has the value u * 2^-24, exactly.  So a K code needs only to
+// be moved into the low bits of a half; the offset that makes it non-negative (u = c + 128
+// for int8, c + 8 for int4) is removed once per score (see the kernel) instead of once per
+// element.
+//
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float pow2f(int e)
+{
+    return __int_as_float((127 + e) << 23);
+}
+
+// Shift e in [-60, 60] that brings x > 0 into [2^13, 2^14) as x * 2^e (60 for x = 0).
+__device__ __forceinline__ int pow2_shift(float x)
+{
+    const int ex = (int)((__float_as_uint(x) >> 23) & 0xffu) - 127;   // x in [2^ex, 2^(ex+1)) if normal
+    return max(-60, min(60, 13 - ex));
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// int8 codes, already XORed with 0x80 (u = c + 128): bytes of w picked by `sel` (nibbles
+// 0..3 pick bytes of w, 4 a zero byte) -> two halves u * 2^-24.
+__device__ __forceinline__ uint32_t u8x2(uint32_t wx, uint32_t sel)
+{
+    return __byte_perm(wx, 0u, sel);
+}
+
+// int4 codes as stored (two's complement nibbles): nibble s (0..3) of each 16-bit half
+// -> two halves.  Even nibbles land in bits 0..3 (u * 2^-24), odd nibbles stay in bits
+// 4..7 (16 u * 2^-24); the XOR that turns c into u = c + 8 rides in the same logic op.
+__device__ __forceinline__ uint32_t u4x2(uint32_t w, int s)
+{
+    const uint32_t x = (s & 2) ? (w >> 8) : w;
+    return (s & 1) ? ((x & 0x00f000f0u) ^ 0x00800080u) : ((x & 0x000f000fu) ^ 0x00080008u);
+}
+
 __device__ __forceinline__ uint32_t h2_sub(uint32_t a, float c)
 {
     __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), __float2half2_rn(c));
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-// int8 codes, already XORed with 0x80 (u = c + 128): two bytes of w chosen by `sel` ->
-// fp16 pair; 0x64XX as fp16 is 1024 + XX.
-__device__ __forceinline__ uint32_t i8x2(uint32_t wx, uint32_t sel)
-{
-    return h2_sub(__byte_perm(wx, 0x64646464u, sel), 1152.f);
-}
-
-// int4 codes, already XORed with 0x8 per nibble (u = c + 8): nibble s (0..3) of each
-// 16-bit half -> fp16 pair.  Even nibbles: 0x640X is 1024 + u; odd nibbles stay in
-// place, 0x64X0 is 1024 + 16 u, and one fused multiply-add by 1/16 removes both biases.
 __device__ __forceinline__ uint32_t h2_fma(uint32_t a, float m, float c)
 {
     __half2 r = __hfma2(*reinterpret_cast<__half2*>(&a), __float2half2_rn(m), __float2half2_rn(c));
     return *reinterpret_cast<uint32_t*>(&r);
 }
 
-__device__ __forceinline__ uint32_t i4x2(uint32_t wx, int s)
+// V codes become NORMAL fp16 integers c: 0x64XX is 1024 + XX, minus 1024 + the offset
+// (exact).  P . V keeps these: P is split into two fp16 parts, and the low part's
+// products with subnormal V codes were measured to lose precision in the tensor cores.
+__device__ __forceinline__ uint32_t i8x2(uint32_t wx, uint32_t sel)
 {
-    const uint32_t w = (s & 2) ? (wx >> 8) : wx;
-    if (s & 1) return h2_fma((w & 0x00f000f0u) | 0x64006400u, 0.0625f, -72.f);
-    return h2_sub((w & 0x000f000fu) | 0x64006400u, 1032.f);
+    return h2_sub(__byte_perm(wx, 0x64646464u, sel), 1152.f);
+}
+
+__device__ __forceinline__ uint32_t i4x2(uint32_t w, int s)
+{
+    const uint32_t x = (s & 2) ? (w >> 8) : w;
+    if (s & 1) return h2_fma(((x & 0x00f000f0u) ^ 0x00800080u) | 0x64006400u, 0.0625f, -72.f);
+    return h2_sub(((x & 0x000f000fu) ^ 0x00080008u) | 0x64006400u, 1032.f);
 }
 
 // e4m3 pair (low byte -> low half) -> fp16 pair.
@@ -145,15 +191,14 @@ __device__ __forceinline__ void kfrag(const uint32_t (&kw)[NW], int ks, uint32_t
 {
     if constexpr (DT == PKV_INT8) {
         const uint32_t w = kw[ks] ^ 0x80808080u;
-        b0 = i8x2(w, 0x4140);
-        b1 = i8x2(w, 0x4342);
+        b0 = u8x2(w, 0x4140);
+        b1 = u8x2(w, 0x4342);
     } else if constexpr (DT == PKV_FP8E4M3) {
         b0 = e4m3x2(kw[ks]);
         b1 = e4m3x2(kw[ks] >> 16);
     } else {
-        const uint32_t w = kw[ks >> 1] ^ 0x88888888u;
-        b0 = i4x2(w, (ks & 1) * 2);
-        b1 = i4x2(w, (ks & 1) * 2 + 1);
+        b0 = u4x2(kw[ks >> 1], (ks & 1) * 2);
+        b1 = u4x2(kw[ks >> 1], (ks & 1) * 2 + 1);
     }
 }
 
@@ -163,8 +208,8 @@ template <int DT>
 __device__ __forceinline__ void vfrags(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t (&va)[4][4])
 {
     if constexpr (DT == PKV_INT4) {
-        const uint32_t ab0 = __byte_perm(a, b, 0x5410) ^ 0x88888888u, ab1 = __byte_perm(a, b, 0x7632) ^ 0x88888888u;
-        const uint32_t cd0 = __byte_perm(c, d, 0x5410) ^ 0x88888888u, cd1 = __byte_perm(c, d, 0x7632) ^ 0x88888888u;
+        const uint32_t ab0 = __byte_perm(a, b, 0x5410), ab1 = __byte_perm(a, b, 0x7632);
+        const uint32_t cd0 = __byte_perm(c, d, 0x5410), cd1 = __byte_perm(c, d, 0x7632);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t ab = j < 2 ? ab0 : ab1, cd = j < 2 ? cd0 : cd1;
@@ -203,6 +248,14 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     using Cfg = QCfg<DT, D>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int ROW = Cfg::ROW, SWZ = Cfg::SWZ;
+    // integer K codes enter Q . K^T as subnormals u * 2^-24 with u = c + OFF; odd int4
+    // nibbles enter as 16 u, and their q is pre-divided by 16.  q is pre-scaled by a power
+    // of two chosen per CTA (largest |q| brought near 2^14) so that the products stay well
+    // clear of the bottom of the accumulator's range; the scaling is exact and is undone,
+    // with the offset, in the score.
+    constexpr bool SUBN = DT != PKV_FP8E4M3;
+    constexpr float OFF = DT == PKV_INT8 ? 128.f : 8.f;
+    constexpr float ODD = DT == PKV_INT4 ? 0.0625f : 1.f;   // q factor on k-slots 8..15
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[STAGES];
 
@@ -265,8 +318,12 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
     }
 
-    // q as fp16 A fragments, k-slots assigned to physical dims by kdim()
+    // q as fp16 A fragments, k-slots assigned to physical dims by kdim(); for integer
+    // codes also -OFF * (sum of the fragments' q over d, odd int4 slots counted times 16)
+    // per head row r, r + 8: the part of 2^24 * (q . k) that the code offset adds
     uint32_t qa[Cfg::KS][4];
+    float qoff[2] = {0.f, 0.f};
+    int eq = 0;   // q is multiplied by 2^eq (integer codes), which brings max |q| to [2^13, 2^14)
     {
         const bool bf = p.q_bf16;
         const uint16_t* qh = static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D;
@@ -275,16 +332,38 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             return bf ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
         };
         const bool r0 = r < GC, r1 = (NHT == 2) && (r + 8 < GC);
+        float qs = 1.f, qo = ODD;
+        if constexpr (SUBN) {
+            float qmax = 0.f;
+            for (int i = lane; i < GC * D; i += 32) qmax = fmaxf(qmax, fabsf(qv(0, i)));
+            eq = pow2_shift(warp_max(qmax));
+            qs = pow2f(eq);
+            qo = qs * ODD;
+        }
 #pragma unroll
         for (int ks = 0; ks < Cfg::KS; ++ks) {
             const int d0 = kdim<DT, D>(ks, qd, 0), d1 = kdim<DT, D>(ks, qd, 1);
             const int d2 = kdim<DT, D>(ks, qd, 2), d3 = kdim<DT, D>(ks, qd, 3);
-            qa[ks][0] = r0 ? pack2<false>(qv(r, d0), qv(r, d1)) : 0u;
-            qa[ks][2] = r0 ? pack2<false>(qv(r, d2), qv(r, d3)) : 0u;
-            qa[ks][1] = r1 ? pack2<false>(qv(r + 8, d0), qv(r + 8, d1)) : 0u;
-            qa[ks][3] = r1 ? pack2<false>(qv(r + 8, d2), qv(r + 8, d3)) : 0u;
+            qa[ks][0] = r0 ? pack2<false>(qv(r, d0) * qs, qv(r, d1) * qs) : 0u;
+            qa[ks][2] = r0 ? pack2<false>(qv(r, d2) * qo, qv(r, d3) * qo) : 0u;
+            qa[ks][1] = r1 ? pack2<false>(qv(r + 8, d0) * qs, qv(r + 8, d1) * qs) : 0u;
+            qa[ks][3] = r1 ? pack2<false>(qv(r + 8, d2) * qo, qv(r + 8, d3) * qo) : 0u;
+        }
+        if constexpr (SUBN) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float even = 0.f, odd = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < Cfg::KS; ++ks) {
+                    const float2 e = unpack2<false>(qa[ks][hr]), o = unpack2<false>(qa[ks][2 + hr]);
+                    even += e.x + e.y;
+                    odd += o.x + o.y;
+                }
+                qoff[hr] = -OFF * pow2f(-eq) * warp_sum_quad(even + odd * (1.f / ODD));
+            }
         }
     }
+    const float kq = pow2f(24 - eq);     // log2-domain score = (acc * 2^(24-eq) + qoff) * sl
 
     float o[Cfg::MT][NHT][4];
 #pragma unroll
@@ -326,18 +405,20 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         }
 
         const float sl = p.scale_log2 * sc_kv.x;
+        const float slk = SUBN ? sl * kq : sl;
         float pr[2][4];
         float alpha[2];
 #pragma unroll
         for (int hr = 0; hr < NHT; ++hr) {
             float x[2][2];
             float mx = -INFINITY;
+            const float cb = SUBN ? qoff[hr] * sl : 0.f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int tok = nt * 8 + 2 * qd + e;
-                    x[nt][e] = (tok < nv && tok >= nlo) ? sc[nt][2 * hr + e] * sl : -INFINITY;
+                    x[nt][e] = (tok < nv && tok >= nlo) ? fmaf(sc[nt][2 * hr + e], slk, cb) : -INFINITY;
                     mx = fmaxf(mx, x[nt][e]);
                 }
             mx = warp_max_quad(mx);
