@@ -386,6 +386,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const uint32_t vb = kb + Cfg::TILE;
         const int nv = min(kBlock, ntok - j * kBlock);
         const int nlo = lo - (tok0 + j * kBlock);   // tokens of this tile before the window: < nlo
+        const bool whole = nv == kBlock && nlo <= 0;   // every token of the tile visible (warp-uniform)
+        // int8 / fp8 skip the score mask on whole tiles; int4 keeps one masked path (its
+        // compiled schedule measured faster that way)
+        constexpr bool SKIP_MASK = DT != PKV_INT4;
         const float2 sc_kv = tsc[j];
 
         // S = Q . K^T, token 8 nt + r of the tile in n-tile nt
@@ -413,14 +417,24 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             float x[2][2];
             float mx = -INFINITY;
             const float cb = SUBN ? qoff[hr] * sl : 0.f;
+            if (SKIP_MASK && whole) {
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int tok = nt * 8 + 2 * qd + e;
-                    x[nt][e] = (tok < nv && tok >= nlo) ? fmaf(sc[nt][2 * hr + e], slk, cb) : -INFINITY;
-                    mx = fmaxf(mx, x[nt][e]);
-                }
+                    for (int e = 0; e < 2; ++e) {
+                        x[nt][e] = fmaf(sc[nt][2 * hr + e], slk, cb);
+                        mx = fmaxf(mx, x[nt][e]);
+                    }
+            } else {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int tok = nt * 8 + 2 * qd + e;
+                        x[nt][e] = (tok < nv && tok >= nlo) ? fmaf(sc[nt][2 * hr + e], slk, cb) : -INFINITY;
+                        mx = fmaxf(mx, x[nt][e]);
+                    }
+            }
             mx = warp_max_quad(mx);
             const float mn = fmaxf(m_run[hr], mx);
             alpha[hr] = ex2(m_run[hr] - mn);
@@ -464,7 +478,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             }
 
         uint32_t keep01 = 0xffffffffu, keep23 = 0xffffffffu;
-        const bool partial = nv < kBlock || nlo > 0;
+        const bool partial = !whole;
         if (partial) {   // zero V outside [nlo, nv): P is 0 there, V may be stale
             auto in = [&](int t) { return t >= nlo && t < nv; };
             keep01 = (in(2 * qd) ? 0x0000ffffu : 0u) | (in(2 * qd + 1) ? 0xffff0000u : 0u);

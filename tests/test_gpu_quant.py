@@ -194,3 +194,45 @@ def test_quantized_long_context_config(dt):
     assert np.array_equal(pool.k_scale[0][idx].cpu().numpy(), opool.k_scale)
     ref = oracle.paged_decode(opool, q[sampled].cpu(), oracle.BF16, sub_t, sub_c, np.float32(d ** -0.5))
     assert max_abs_diff(out[sampled], ref) <= TOL
+
+
+# q magnitudes: the integer-code kernels pre-scale q by a power of two chosen per CTA
+# from its largest |q| (and treat all-zero q separately); the fp8 kernel does not.
+Q_MAGNITUDES = {
+    "zero": lambda q: q * 0,                 # every score 0: out = mean of the dequantized V
+    "tiny": lambda q: q * 1e-3,              # q near the bottom of fp16's normal range
+    "large": lambda q: q * 4,                # peaked softmax
+    "mixed": lambda q: q * torch.where(torch.arange(q.shape[1]) % 4 == 0, 4.0, 0.01)[None, :, None],
+}
+
+
+@pytest.mark.parametrize("mag", list(Q_MAGNITUDES))
+@pytest.mark.parametrize("dt", QDTYPES, ids=lambda x: NAMES[x])
+def test_quantized_decode_query_magnitudes(dt, mag):
+    H_q, H_kv, d = 32, 4, 128
+    g = wl.generator(1200 + 10 * dt + list(Q_MAGNITUDES).index(mag))
+    lens = [1, 16, 40] + torch.randint(100, 400, (3,), generator=g).tolist()
+    N = sum(wl.ceil_div(n, 16) for n in lens) + 2
+    paging = wl.allocate(lens, N, 32, g)
+    pool = pkv.KVPool.allocate(1, N, H_kv, d, dt)
+    seq = torch.cat([torch.full((n,), b) for b, n in enumerate(lens)])
+    pos = torch.cat([torch.arange(n) for n in lens])
+    slots = wl.slots_for(paging.tables, seq, pos)
+    k, v = wl.kv_source(len(seq), H_kv, d, g, outliers=wl.outlier_channels(g, H_kv, d))
+    pkv.kv_append(pool, 0, k.to(DEV), v.to(DEV), slots.to(DEV))
+    opool = oracle_copy(pool)
+    q = Q_MAGNITUDES[mag](wl.normal((len(lens), H_q, d), torch.float32, g)).to(torch.bfloat16)
+    out = pkv.paged_decode_attn(pool, 0, q.to(DEV), paging.tables.to(DEV), paging.ctx_lens.to(DEV), d ** -0.5,
+                                max(lens))
+    torch.cuda.synchronize()
+    assert pkv.read_device_status(pool) == 0
+    ref = oracle.paged_decode(opool, q, oracle.BF16, paging.tables, paging.ctx_lens, np.float32(d ** -0.5))
+    assert max_abs_diff(out, ref) <= TOL
+    if mag == "zero":   # closed form: uniform weights, out = mean of each sequence's V rows
+        vdq = opool.dequant("v")
+        G = H_q // H_kv
+        for b, n in enumerate(lens):
+            t = np.arange(n)
+            rows = vdq[paging.tables[b].numpy()[t // 16], :, t % 16, :]      # [n, H_kv, d]
+            want = np.repeat(rows.mean(axis=0), G, axis=0)                     # [H_q, d]
+            assert np.abs(out[b].cpu().double().numpy() - want).max() <= TOL
