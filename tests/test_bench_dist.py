@@ -72,3 +72,21 @@ def test_reference_arm_under_torchrun_prints_from_rank_zero_only():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["unit"] == "GB/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_clock_summary_of_nvidia_smi_rows():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    rows = [
+        "0, 1965, 1965, 650.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1770, 1965, 998.7, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 990.0, 0x0, Not Active, Not Active, Not Active, Not Active",   # unparsable: skipped
+        "garbage",
+    ]
+    got = bench.summarize_clocks(rows)
+    assert got == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    slow = bench.summarize_clocks(["0, 1500, 1965, 700, 0x8, Active, Not Active, Active, Not Active"])
+    assert slow["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarize_clocks([]) is None
