@@ -170,3 +170,49 @@ def test_block_moves_validate_on_the_host():
         assert L.kv_swap_in(h, fake, 1, ctypes.c_void_p(ctypes.addressof(buf) + 8), None) == -2
     finally:
         L.kv_pool_destroy(h)
+
+
+def _decode_ws(h, B, H_q, ctx, opts=None):
+    return pkv.lib().paged_decode_workspace_bytes(h, B, H_q, ctx, ctypes.byref(opts) if opts is not None else None)
+
+
+@pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 1024), (pkv.FP8E4M3, 1024),
+                                     (pkv.INT4, 2048)])
+def test_decode_workspace_follows_the_partition_policy(dtype, P):
+    """Split-K partitions of ~256 KiB of K + V whatever the storage dtype (512 / 1024 / 2048 tokens at
+    d = 128) when the batch fills the GPU; the workspace is fp32 o[d] + (m, l) per (sequence, query
+    head, partition)."""
+    kw = dict(num_kv_heads=8, head_dim=128, kv_dtype=dtype)
+    if dtype in pkv.QUANTIZED:
+        kw.update(k_scale=0x30000, v_scale=0x40000)
+    rc, h = _create(**kw)
+    assert rc == 0
+    try:
+        B, H_q, ctx = 170, 64, 8192
+        assert _decode_ws(h, B, H_q, ctx) == B * H_q * (-(-ctx // P)) * (128 + 2) * 4
+        # a context of one default partition: with only B * H_kv CTAs the grid cannot fill the GPU, so
+        # partitions are halved (to 128 tokens at least) and the partials come back
+        short = _decode_ws(h, B, H_q, P)
+        parts, rem = divmod(short, B * H_q * (128 + 2) * 4)
+        assert rem == 0 and 2 <= parts <= P // 128 and parts & (parts - 1) == 0
+        assert _decode_ws(h, B, H_q, 128) == 0                         # one partition: no partials
+    finally:
+        pkv.lib().kv_pool_destroy(h)
+
+
+def test_decode_workspace_small_batches_and_explicit_partitions():
+    rc, h = _create(num_kv_heads=8, head_dim=128, kv_dtype=pkv.BF16)
+    assert rc == 0
+    try:
+        row = (128 + 2) * 4
+        # 2 sequences cannot fill 148 SMs with 512-token partitions: they shrink to the 128-token floor
+        assert _decode_ws(h, 2, 64, 8192) == 2 * 64 * 64 * row
+        # an explicit partition size is taken as given (a multiple of 16 in [64, 4096])
+        assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, 64, 0)) == 3 * 16 * 16 * row
+        assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, 4096, 0)) == 0
+        for bad in (100, 48, 8192):
+            assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, bad, 0)) == 0
+        # the partials scale with the batch and the query heads, not with the KV heads' grouping
+        assert _decode_ws(h, 340, 64, 8192) == 2 * _decode_ws(h, 170, 64, 8192)
+    finally:
+        pkv.lib().kv_pool_destroy(h)
