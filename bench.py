@@ -667,6 +667,12 @@ def run_gpu(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_oracle(args.workload, budget_s=args.cpu_seconds)
+        try:
+            every = cpu_oracle_all_cores(args.workload, budget_s=args.cpu_seconds / 2)
+        except Exception as e:   # the all-cores figure is extra; never lose the line over it
+            every = {"error": repr(e)}
+        if every is not None:
+            res["cpu_baseline"]["all_cores"] = every
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:
@@ -730,6 +736,88 @@ def cpu_oracle(workload, budget_s=12.0, per_step=None, steps=None, warmup=0):
            "sample": f"{seqs} whole sequence(s) of one layer of the {workload} workload ({total_tok} cached "
                      f"tokens), fp64 C oracle, single thread, {total_s:.1f} s"}
     return (res, step_secs) if per_step else res
+
+
+def cpu_oracle_all_cores(workload, budget_s=6.0, max_threads=64, mem_budget=8e9):
+    """The same oracle calls from T concurrent host threads (ctypes releases the GIL while the C
+    oracle runs), one whole sequence of the workload per thread; T = the cores this process may
+    run on, capped by `max_threads` and by a host-memory budget.  Aggregate K/V bytes of the
+    completed calls over the wall time from the common start until the last call in flight at
+    `budget_s` ends.
+    Returns None for the block-move workload, or a dict with an "error" key if a thread failed."""
+    import threading
+
+    import oracle
+
+    cfg = WORKLOADS[workload]
+    if cfg["kind"] == "blocks":
+        return None
+    oracle.build()
+    oracle.lib()
+    H_q, H_kv, d, dt = cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
+    gen = wl.generator(431 + 3)
+    if cfg["kind"] == "prefix":
+        ctx = (4000 + 200 + torch.randint(0, 301, (cfg["B"],), generator=gen, dtype=torch.int32) + 1)
+    else:
+        ctx = make_lens(cfg["lens"], gen, cfg["B"])
+    quant = dt in (wl.INT8, wl.FP8, wl.INT4)
+    window = cfg.get("window", 0)
+    # host bytes per thread: the oracle's pool plus the bf16 K and V source it is built from
+    per_seq = float(ctx.float().max()) * H_kv * d * (2 * ELEM_BYTES[dt] + 4)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    T = max(1, min(cores, max_threads, int(mem_budget // per_seq)))
+    stop = threading.Event()
+    start = threading.Barrier(T + 1, timeout=600)
+    done_bytes = [0] * T
+    errors = []
+
+    def worker(i):
+        try:
+            n = int(ctx[i % len(ctx)])
+            g = wl.generator(431 + 700 + i)
+            nb = wl.ceil_div(n, 16)
+            table = torch.arange(nb, dtype=torch.int32).view(1, nb)
+            opool = oracle.Pool(nb, H_kv, d, dt)
+            k, v = wl.kv_source(n, H_kv, d, g) if quant else (wl.normal((n, H_kv, d), torch.bfloat16, g),
+                                                             wl.normal((n, H_kv, d), torch.bfloat16, g))
+            oracle.kv_append(opool, k, v, oracle.BF16, np.arange(n, dtype=np.int32))
+            del k, v
+            q = wl.normal((1, H_q, d), torch.bfloat16, g)
+            seen = min(n, window) if window else n
+            start.wait()
+            while not stop.is_set():
+                oracle.paged_decode(opool, q, oracle.BF16, table, [n], np.float32(d ** -0.5), window=window)
+                done_bytes[i] += seen * 2 * H_kv * d * ELEM_BYTES[dt]
+        except Exception as e:   # a failed thread ends the measurement, not the bench
+            errors.append(repr(e))
+            start.abort()
+
+    prev_threads = torch.get_num_threads()
+    torch.set_num_threads(1)   # one host core per oracle thread, also while generating
+    threads = [threading.Thread(target=worker, args=(i,), daemon=True) for i in range(T)]
+    try:
+        for t in threads:
+            t.start()
+        try:
+            start.wait()
+        except threading.BrokenBarrierError:
+            stop.set()
+            return {"error": errors[0] if errors else "threads did not start"}
+        t0 = time.perf_counter()
+        time.sleep(budget_s)
+        stop.set()
+        for t in threads:
+            t.join(timeout=600)
+        wall = time.perf_counter() - t0
+    finally:
+        stop.set()
+        torch.set_num_threads(prev_threads)
+    if errors or any(t.is_alive() for t in threads):
+        return {"error": errors[0] if errors else "a thread did not finish"}
+    total = sum(done_bytes)
+    return {"value": round(total / wall / 1e9, 4), "unit": "GB/s", "cores": T,
+            "sample": f"{T} threads, one whole sequence of one layer each, fp64 C oracle called concurrently; "
+                      f"{total / 1e9:.2f} GB of K/V in {wall:.1f} s"}
 
 
 def cpu_oracle_blocks(cfg, workload, budget_s, per_step=None, steps=None, warmup=0):

@@ -90,3 +90,21 @@ def test_clock_summary_of_nvidia_smi_rows():
     slow = bench.summarize_clocks(["0, 1500, 1965, 700, 0x8, Active, Not Active, Active, Not Active"])
     assert slow["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.summarize_clocks([]) is None
+
+
+def test_all_cores_oracle_timing_on_host_threads(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+
+    got = bench.cpu_oracle_all_cores("llama8b", budget_s=0.5, max_threads=2)
+    assert set(got) == {"value", "unit", "cores", "sample"}
+    assert got["value"] > 0 and got["unit"] == "GB/s" and 1 <= got["cores"] <= 2
+    assert bench.cpu_oracle_all_cores("blocks") is None
+
+    def broken(*a, **k):
+        raise RuntimeError("planted failure")
+
+    monkeypatch.setattr(oracle, "paged_decode", broken)   # a failing thread ends the measurement, not the bench
+    bad = bench.cpu_oracle_all_cores("llama8b", budget_s=0.5, max_threads=2)
+    assert "planted failure" in bad["error"]
