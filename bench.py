@@ -820,6 +820,87 @@ def cpu_oracle_all_cores(workload, budget_s=6.0, max_threads=64, mem_budget=8e9)
                       f"{total / 1e9:.2f} GB of K/V in {wall:.1f} s"}
 
 
+def cpu_oracle_waves(workload, steps, warmup, max_threads=64, mem_budget=8e9):
+    """--impl reference on the host's cores: each step is one wave of T whole sequences of one
+    layer, one per host thread (T = the cores this process may run on, capped by `max_threads`
+    and a host-memory budget), the C oracle called concurrently (ctypes releases the GIL).  A
+    step's time runs from the moment every thread holds its generated sequence until the last
+    call returns.  Returns (result dict, list of per-step seconds)."""
+    import threading
+
+    import oracle
+
+    cfg = WORKLOADS[workload]
+    oracle.build()
+    oracle.lib()
+    H_q, H_kv, d, dt = cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
+    gen = wl.generator(431 + 3)
+    if cfg["kind"] == "prefix":
+        ctx = (4000 + 200 + torch.randint(0, 301, (cfg["B"],), generator=gen, dtype=torch.int32) + 1)
+    else:
+        ctx = make_lens(cfg["lens"], gen, cfg["B"])
+    quant = dt in (wl.INT8, wl.FP8, wl.INT4)
+    window = cfg.get("window", 0)
+    per_seq = float(ctx.float().max()) * H_kv * d * (2 * ELEM_BYTES[dt] + 4)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    T = max(1, min(cores, max_threads, int(mem_budget // per_seq)))
+    step_secs, total_kv, total_tok = [], 0, 0
+    prev_threads = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        for s in range(warmup + steps):
+            ready = threading.Barrier(T + 1, timeout=900)
+            finished = threading.Barrier(T + 1, timeout=900)
+            seen = [0] * T
+            errors = []
+
+            def worker(i):
+                try:
+                    sid = (s * T + i) % len(ctx)
+                    n = int(ctx[sid])
+                    g = wl.generator(431 + 900 + s * T + i)
+                    nb = wl.ceil_div(n, 16)
+                    table = torch.arange(nb, dtype=torch.int32).view(1, nb)
+                    opool = oracle.Pool(nb, H_kv, d, dt)
+                    k, v = wl.kv_source(n, H_kv, d, g) if quant else (wl.normal((n, H_kv, d), torch.bfloat16, g),
+                                                                     wl.normal((n, H_kv, d), torch.bfloat16, g))
+                    oracle.kv_append(opool, k, v, oracle.BF16, np.arange(n, dtype=np.int32))
+                    del k, v
+                    q = wl.normal((1, H_q, d), torch.bfloat16, g)
+                    ready.wait()
+                    oracle.paged_decode(opool, q, oracle.BF16, table, [n], np.float32(d ** -0.5), window=window)
+                    seen[i] = min(n, window) if window else n
+                    finished.wait()
+                except Exception as e:
+                    errors.append(repr(e))
+                    ready.abort()
+                    finished.abort()
+
+            threads = [threading.Thread(target=worker, args=(i,), daemon=True) for i in range(T)]
+            for t in threads:
+                t.start()
+            ready.wait()
+            t0 = time.perf_counter()
+            finished.wait()
+            dt_s = time.perf_counter() - t0
+            for t in threads:
+                t.join(timeout=60)
+            if errors:
+                raise RuntimeError(errors[0])
+            if s >= warmup:
+                step_secs.append(dt_s)
+                total_tok += sum(seen)
+                total_kv += sum(seen) * 2 * H_kv * d * ELEM_BYTES[dt]
+    finally:
+        torch.set_num_threads(prev_threads)
+    total_s = sum(step_secs)
+    res = {"value": round(total_kv / total_s / 1e9, 4), "unit": "GB/s", "cores": T, "kind": "oracle",
+           "seq_tokens_per_s_per_layer": round(total_tok / total_s),
+           "sample": f"{steps} step(s) of {T} whole sequences of one layer of the {workload} workload, one per "
+                     f"host thread, fp64 C oracle called concurrently ({total_tok} cached tokens, {total_s:.1f} s)"}
+    return res, step_secs
+
+
 def cpu_oracle_blocks(cfg, workload, budget_s, per_step=None, steps=None, warmup=0):
     """The oracle's block copy (numpy byte moves, every layer) on a bounded sample of pairs
     from a small pool of the same shape."""
@@ -857,12 +938,17 @@ def cpu_oracle_blocks(cfg, workload, budget_s, per_step=None, steps=None, warmup
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle on this host, same workload, metric and unit;
-    each step is a bounded sample (--ref-seqs whole sequences of one layer)."""
+    """--impl reference: the CPU oracle on this host's cores, same workload, metric and unit;
+    each step is a bounded sample: one wave of whole sequences of one layer, one per host
+    thread (--ref-threads 1: --ref-seqs sequences on one thread)."""
     rank, _, world = dist_env()
     if rank != 0:
         return
-    cpu, secs = cpu_oracle(args.workload, per_step=max(1, args.ref_seqs), steps=args.steps, warmup=args.warmup)
+    if args.ref_threads == 1 or WORKLOADS[args.workload]["kind"] == "blocks":
+        cpu, secs = cpu_oracle(args.workload, per_step=max(1, args.ref_seqs), steps=args.steps, warmup=args.warmup)
+    else:
+        cpu, secs = cpu_oracle_waves(args.workload, steps=args.steps, warmup=args.warmup,
+                                     max_threads=args.ref_threads if args.ref_threads > 0 else 64)
     res = {"metric": METRIC, "value": cpu["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 2), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None,
@@ -885,7 +971,11 @@ def main():
     ap.add_argument("--pool-fraction", type=float, default=0.4,
                     help="fraction of free HBM used for distinct per-layer pools")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-seqs", type=int, default=2)
+    ap.add_argument("--ref-seqs", type=int, default=2,
+                    help="--impl reference with --ref-threads 1: whole sequences per step")
+    ap.add_argument("--ref-threads", type=int, default=0,
+                    help="--impl reference: host threads calling the oracle concurrently, one sequence "
+                         "each per step (0: every usable core, at most 64; 1: one thread)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--partition", type=int, default=0,
                     help="split-K partition size in tokens (0: chosen by the library)")
