@@ -229,10 +229,11 @@ class Timed:
 def build_decode(args, cfg, dev, rank):
     from paged_kv_cache_431_b200 import pkv
 
-    L, B, H_q, H_kv, d, dt = cfg["layers"], cfg["B"], cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
+    L, H_q, H_kv, d, dt = cfg["layers"], cfg["H_q"], cfg["H_kv"], cfg["d"], cfg["dtype"]
+    B = args.batch or cfg["B"]
     gen = wl.generator(431 + 3 + rank)
     ctx = make_lens(cfg["lens"], gen, B)
-    N = cfg["pool_blocks"]
+    N = cfg["pool_blocks"] * B // cfg["B"]   # the pool scales with a --batch override
     paging = wl.allocate(ctx, N, cfg["width"], gen)
     quant = dt in (wl.INT8, wl.FP8, wl.INT4)
     per_layer_pool = 2 * N * H_kv * 16 * d * ELEM_BYTES[dt]
@@ -290,8 +291,10 @@ def build_decode(args, cfg, dev, rank):
                 ev[l][1].record(stream)
 
     kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt, window)
+    # this library's kernels per layer: the append (3 for quantized pools) and the decode (its split-K
+    # merge is fused into it; the CUDA-core engines launch a separate merge)
     parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, sliding_window=window) > 0
-    launches = L * ((3 if quant else 1) + 1 + (1 if parts else 0))
+    launches = L * ((3 if quant else 1) + 1 + (1 if parts and args.engine in (2, 3) else 0))
 
     # host-buffer (e2e) step: inputs from pinned memory, every layer's output read back
     g = wl.generator(999)
@@ -345,10 +348,15 @@ def build_decode(args, cfg, dev, rank):
     d2h_bytes = hout.numel() * hout.element_size()
     peaks, kind = measured_peaks()
     info = dict(
-        config={"workload": args.workload, "description": cfg["desc"], "layers": L, "batch": B, "q_heads": H_q,
+        config={"workload": args.workload if B == cfg["B"] else f"{args.workload} (batch {B})",
+                "description": cfg["desc"], "layers": L, "batch": B, "q_heads": H_q,
                 "kv_heads": H_kv, "head_dim": d, "kv_dtype": DTYPE_NAME[dt], "sum_ctx": int(ctx.sum()),
                 "physical_layer_pools": L_phys, "parallelism": "replicas",
-                "l2": f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V",
+                "l2": (f"inputs larger than L2: each decode call reads {kv / 1e9:.2f} GB of K/V from one of "
+                       f"{L_phys} layer pools" if L > 1 else
+                       f"L2 flushed between timed steps (a 256 MiB write, then a read of it, outside the timed "
+                       f"events); each decode "
+                       f"call reads {kv / 1e9:.2f} GB of K/V"),
                 "partition_tokens": args.partition or "auto", "sliding_window": window or None,
                 "decode_engine": {0: "tensor cores (mma.sync)", 1: "tensor cores (mma.sync)",
                                   2: "CUDA cores, packed fp32x2 FMA", 3: "CUDA cores, fp32 FMA"}[args.engine]},
@@ -359,7 +367,7 @@ def build_decode(args, cfg, dev, rank):
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
                       traffic=kernel_traffic(f"decode_{args.workload}", DECODEQ_SRCS if quant else DECODE16_SRCS)),
         launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",
-        h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L)
+        h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L, flush_l2=L == 1)
     return step, e2e_step, info, pool
 
 
@@ -553,24 +561,53 @@ def job_throughput(units_per_step: float, steps: int, world: int, elapsed_ms: fl
     return units_per_step * steps * world / (elapsed_ms * 1e-3)
 
 
-def time_steps(step, n_steps, per_step_calls, dev, world):
+def time_steps(step, n_steps, per_step_calls, dev, world, flush=None):
+    """Device time of n_steps steps (CUDA events on the launching stream).  With `flush`, it
+    runs before every step outside the timed events (an L2 flush), and the time is the sum of
+    the steps' own event intervals."""
     timed = Timed(n_steps, per_step_calls)
     stream = torch.cuda.current_stream(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for s in range(n_steps):
-        step(timed.ev[s] if timed is not None else None)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1)
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    if flush is None:
+        t0, t1 = mk(), mk()
+        t0.record(stream)
+        for s in range(n_steps):
+            step(timed.ev[s])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = t0.elapsed_time(t1)
+    else:
+        marks = [(mk(), mk()) for _ in range(n_steps)]
+        for s in range(n_steps):
+            flush()
+            marks[s][0].record(stream)
+            step(timed.ev[s])
+            marks[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(a.elapsed_time(b) for a, b in marks)
     if world > 1:
         torch.distributed.barrier()
         ms = max_over_ranks(ms, dev)
     return ms, timed
+
+
+class L2Flush:
+    """Writes a buffer twice the size of the L2 (126 MB on B200), so no input of the next step
+    is still cached, then reads it back: the L2 is left holding clean lines, so the timed step
+    does not also pay for writing the flush's dirty lines back to HBM."""
+
+    def __init__(self, dev, nbytes=256 << 20):
+        self.buf = torch.empty(nbytes // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int64, device=dev)
+        self.n = 0
+
+    def __call__(self):
+        self.n += 1
+        self.buf.fill_(self.n)
+        torch.sum(self.buf, dtype=torch.int64, out=self.sink)
 
 
 def run_gpu(args):
@@ -600,14 +637,17 @@ def run_gpu(args):
             graph.replay()
         torch.cuda.synchronize(dev)
 
+    # single-layer decode workloads re-read inputs that could still sit in L2 from the step
+    # before: flush it between timed steps (the 80-layer step cycles over pools >> L2)
+    flush = L2Flush(dev) if info.get("flush_l2") else None
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
     # per-call durations (the roofline) from eager steps with events around each call
-    eager_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world)
+    eager_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world, flush)
     elapsed_ms = eager_ms
     if graph is not None:
-        elapsed_ms, _ = time_steps(lambda ev=None: graph.replay(), args.steps, 1, dev, world)
+        elapsed_ms, _ = time_steps(lambda ev=None: graph.replay(), args.steps, 1, dev, world, flush)
     clk = clocks.stop()
     if pkv.read_device_status(pool):
         raise RuntimeError("device status set during timing")
@@ -618,7 +658,7 @@ def run_gpu(args):
     for _ in range(max(1, args.warmup)):
         e2e_step()
     torch.cuda.synchronize(dev)
-    e2e_ms, _ = time_steps(lambda ev=None: e2e_step(), args.steps, 1, dev, world)
+    e2e_ms, _ = time_steps(lambda ev=None: e2e_step(), args.steps, 1, dev, world, flush)
 
     ms_per_step = elapsed_ms / args.steps
     value = job_throughput(info["kv_bytes_per_step"], args.steps, world, elapsed_ms) / 1e9
@@ -879,14 +919,17 @@ def cpu_oracle_waves(workload, steps, warmup, max_threads=64, mem_budget=8e9):
             threads = [threading.Thread(target=worker, args=(i,), daemon=True) for i in range(T)]
             for t in threads:
                 t.start()
-            ready.wait()
-            t0 = time.perf_counter()
-            finished.wait()
-            dt_s = time.perf_counter() - t0
+            try:   # a failed worker aborts both barriers: report its own exception, not the barrier's
+                ready.wait()
+                t0 = time.perf_counter()
+                finished.wait()
+                dt_s = time.perf_counter() - t0
+            except threading.BrokenBarrierError:
+                dt_s = None
             for t in threads:
                 t.join(timeout=60)
-            if errors:
-                raise RuntimeError(errors[0])
+            if errors or dt_s is None:
+                raise RuntimeError(errors[0] if errors else "a host thread did not reach the barrier")
             if s >= warmup:
                 step_secs.append(dt_s)
                 total_tok += sum(seen)
@@ -983,6 +1026,9 @@ def main():
                     help="prefix_chunk: decode the shared-prefix batch in the cascade form or plainly")
     ap.add_argument("--graph", type=int, default=1, choices=[0, 1],
                     help="1: time the device-resident steps as replays of one CUDA-graph-captured step")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="decode workloads: sequences per call instead of the workload's own batch (small "
+                         "cases for profiler captures; the JSON line is then not the named workload)")
     ap.add_argument("--engine", type=int, default=0, choices=[0, 1, 2, 3],
                     help="decode engine: 0/1 tensor cores, 2 CUDA-core packed FMA, 3 CUDA-core FMA")
     args = ap.parse_args()

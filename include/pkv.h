@@ -22,7 +22,8 @@
  *     library allocates only the small host-side pool handle.  Pointers marked [device]
  *     must be device pointers; [host] are host pointers.
  *   - Calls are asynchronous on the given stream (a cudaStream_t passed as void*; NULL is
- *     the legacy default stream) and never synchronize, except pkv_read_device_status.
+ *     the legacy default stream) and never synchronize, except pkv_read_device_status
+ *     (pkv_get_device_status).
  *   - Every call validates its arguments on the host before any launch and returns
  *     PKV_OK (0) or a negative PKV_ERR_* code; on error nothing is launched.
  *   - Errors only the device can see (a block id outside the pool, a slot outside the
@@ -49,6 +50,7 @@ extern "C" {
 #endif
 
 #define PKV_BLOCK_SIZE 16
+#define PKV_MAX_LAYERS 256   /* layers a pool handle may describe */
 
 /* storage / input dtypes */
 #define PKV_F16     0
@@ -86,7 +88,8 @@ typedef struct pkv_pool* pkv_pool_t;   /* opaque host-side handle */
  * k_scale, v_scale [device]: [num_layers][num_blocks][num_kv_heads] fp32, required for
  * quantized dtypes, ignored otherwise.  device_status [device]: optional int32 word
  * (NULL disables device error reporting); the caller zeroes it before first use.
- * Base pointers must be 16-byte aligned.  Supported: block_size 16, head_dim 64 or 128.
+ * Base pointers must be 16-byte aligned.  Supported: block_size 16, head_dim 64 or 128,
+ * 1 .. PKV_MAX_LAYERS layers.  Layers in separate allocations: kv_pool_create_layers.
  */
 typedef struct {
     int32_t num_layers;
@@ -112,6 +115,21 @@ PKV_API size_t pkv_pool_bytes(const pkv_pool_desc* desc, size_t* scale_bytes);
  * for the cache").  The pool memory stays owned by the caller and must outlive the
  * handle.  *out [host] receives the handle.  No CUDA call is made. */
 PKV_API int kv_pool_create(const pkv_pool_desc* desc, pkv_pool_t* out);
+
+/*
+ * kv_pool_create_layers -- kv_pool_create for a cache whose layers live in separate
+ * allocations (an engine that allocates each layer's cache on its own: the memory equation
+ * of [KVG] "Mechanics" is per layer).  desc gives the geometry, dtype and status word; its
+ * k_data, v_data, k_scale and v_scale are ignored (they may be NULL).
+ *   k_layers, v_layers [host arrays of num_layers device pointers]: layer l's K and V pools,
+ *     each [num_blocks][num_kv_heads][16][row_bytes], 16-byte aligned.
+ *   k_scale_layers, v_scale_layers [host arrays of num_layers device pointers]: layer l's
+ *     fp32 scales [num_blocks][num_kv_heads] (quantized dtypes; NULL arrays otherwise).
+ * The arrays are copied into the handle; the memory they point to stays the caller's.
+ * Every call then works on the handle as on a dense pool.  No CUDA call is made.
+ */
+PKV_API int kv_pool_create_layers(const pkv_pool_desc* desc, void* const* k_layers, void* const* v_layers,
+                                  float* const* k_scale_layers, float* const* v_scale_layers, pkv_pool_t* out);
 
 /* Release a handle (not the pool memory).  NULL is accepted. */
 PKV_API int kv_pool_destroy(pkv_pool_t pool);
@@ -152,7 +170,7 @@ typedef struct {
                                   16-bit pools, head_dim 128, G 4 or 8, q 16-byte aligned (else
                                   PKV_ERR_UNSUPPORTED); kept to measure the FP32-pipe form of the decode */
     int32_t partition_tokens;  /* tokens per split-K partition; 0 = chosen from the workload; else a
-                                  multiple of 16 in [64, 16384] */
+                                  multiple of 16 in [64, 4096] (PKV_ERR_ARG otherwise) */
     int32_t sliding_window;    /* 0 = attend to the whole context; w > 0 = sliding-window attention
                                   ([KVB] "The KV cache": sliding-window or local attention layers):
                                   the query (position context_len - 1) sees only positions
@@ -161,8 +179,10 @@ typedef struct {
 } pkv_decode_opts;
 
 /* Workspace paged_decode_attn needs for these sizes and options (bytes): per (sequence,
- * query head, partition) a head_dim + 2 fp32 partial (o, m, l).  With a sliding window the
- * partitions cover at most window + 15 tokens per sequence. */
+ * query head, partition) a head_dim + 2 fp32 partial (o, m, l), then one int32 merge counter
+ * per (sequence, KV head, group of 16 query heads), which every call clears itself (one
+ * cudaMemsetAsync); 0 when every sequence fits one partition.
+ * With a sliding window the partitions cover at most window + 15 tokens per sequence. */
 PKV_API size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads,
                                     int max_context_len, const pkv_decode_opts* opts);
 
@@ -209,8 +229,8 @@ PKV_API int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_d
  * The first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture on the device.
  * All calls share the buffer and it keeps the last call's contents (no call relies on them:
- * each writes every partial it reads).  Calls whose kernels may overlap on the GPU race on
- * the buffer; issue them in order on one stream.
+ * each writes every partial it reads and clears the merge counters it uses).  Calls whose
+ * kernels may overlap on the GPU race on the buffer; issue them in order on one stream.
  */
 PKV_API int paged_decode_attn_noalloc(pkv_pool_t pool, int layer, const void* q, int q_dtype,
                                       const int32_t* block_tables, int block_table_width,
@@ -323,9 +343,27 @@ PKV_API int kv_swap_out(pkv_pool_t pool, const int32_t* blocks, int num_blocks_t
 PKV_API int kv_swap_in(pkv_pool_t pool, const int32_t* blocks, int num_blocks_to_move, const void* host, void* stream);
 
 /* Synchronize `stream`, read and clear the pool's device status word.  *status_out [host]
- * receives the PKV_DEV_* bits (0 if the pool has no status word).  Returns PKV_ERR_INDEX
- * or PKV_ERR_TIMEOUT if bits were set, PKV_OK otherwise. */
+ * receives the PKV_DEV_* bits (0 if the pool has no status word).  Returns PKV_ERR_TIMEOUT
+ * if PKV_DEV_TIMEOUT was set, else PKV_ERR_INDEX if other bits were set, PKV_OK otherwise. */
 PKV_API int pkv_read_device_status(pkv_pool_t pool, void* stream, int32_t* status_out);
+
+/* The same call under the name pkv_get_device_status. */
+PKV_API int pkv_get_device_status(pkv_pool_t pool, void* stream, int32_t* status_out);
+
+/*
+ * pkv_test_withhold_copy -- a test hook for the bounded waits of the attention kernels (the
+ * pages have no counterpart; it exists so that the path a kernel takes when a bulk copy never
+ * lands can be exercised without faulting anything).  With tile >= 0, every attention kernel
+ * launched afterwards in this process (paged_decode_attn and its variants, the prefill
+ * chunk, the cascade prefix pass) arms the barrier of its tile-th K/V tile (counted per CTA
+ * from 0) without issuing the copy, so that wait never completes, and bounds every wait at
+ * wait_cycles SM clock cycles (1 .. 2e9) instead of about 1 s.  A CTA that gives up sets
+ * PKV_DEV_TIMEOUT, waits (bounded) for the copies it did issue and for its tensor-core work,
+ * and returns without writing its outputs; nothing traps.  tile < 0 restores the defaults
+ * (no tile withheld, waits of about 1 s).  Process-wide, not synchronized with launches in
+ * flight: for tests only.  Returns PKV_ERR_ARG for wait_cycles out of range.
+ */
+PKV_API int pkv_test_withhold_copy(int tile, long long wait_cycles);
 
 /* A static description of a status code. */
 PKV_API const char* pkv_strerror(int status);

@@ -4,6 +4,7 @@
 // pkv_read_device_status.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 #include <new>
 
@@ -11,6 +12,16 @@
 #include "../../include/pkv_block_manager.h"
 
 namespace pkv {
+
+namespace {
+std::atomic<int> g_hold_tile{-1};
+std::atomic<long long> g_wait_cycles{kDefaultWaitCycles};
+}  // namespace
+
+WaitHook wait_hook()
+{
+    return WaitHook{g_hold_tile.load(std::memory_order_relaxed), g_wait_cycles.load(std::memory_order_relaxed)};
+}
 
 int row_bytes_of(int dtype, int head_dim)
 {
@@ -78,10 +89,8 @@ int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtenso
         pool->tmk.resize(L);
         pool->tmv.resize(L);
         for (int l = 0; l < L; ++l) {
-            uint8_t* kb = static_cast<uint8_t*>(pool->d.k_data) + (size_t)l * pool->layer_bytes;
-            uint8_t* vb = static_cast<uint8_t*>(pool->d.v_data) + (size_t)l * pool->layer_bytes;
-            if (!make_map(&pool->tmk[l], kb, pool->d, pool->row_bytes) ||
-                !make_map(&pool->tmv[l], vb, pool->d, pool->row_bytes))
+            if (!make_map(&pool->tmk[l], pool->k_base[l], pool->d, pool->row_bytes) ||
+                !make_map(&pool->tmv[l], pool->v_base[l], pool->d, pool->row_bytes))
                 return PKV_ERR_CUDA;
         }
         pool->maps_ready = true;
@@ -141,7 +150,8 @@ const char* pkv_strerror(int status)
 static int validate_desc(const pkv_pool_desc* d)
 {
     if (!d) return PKV_ERR_NULL;
-    if (d->num_layers <= 0 || d->num_blocks <= 0 || d->num_kv_heads <= 0) return PKV_ERR_ARG;
+    if (d->num_layers <= 0 || d->num_layers > PKV_MAX_LAYERS || d->num_blocks <= 0 || d->num_kv_heads <= 0)
+        return PKV_ERR_ARG;
     if (d->block_size != PKV_BLOCK_SIZE) return PKV_ERR_ARG;
     if (d->head_dim != 64 && d->head_dim != 128) return PKV_ERR_UNSUPPORTED;
     if (row_bytes_of(d->kv_dtype, d->head_dim) <= 0) return PKV_ERR_DTYPE;
@@ -159,6 +169,37 @@ size_t pkv_pool_bytes(const pkv_pool_desc* d, size_t* scale_bytes)
     return per_layer * d->num_layers;
 }
 
+// A handle over per-layer bases (validated by the caller), or null when out of memory.
+static pkv_pool* new_pool(const pkv_pool_desc* d, void* const* k, void* const* v, float* const* ks, float* const* vs)
+{
+    pkv_pool* p = new (std::nothrow) pkv_pool();
+    if (!p) return nullptr;
+    p->d = *d;
+    p->row_bytes = row_bytes_of(d->kv_dtype, d->head_dim);
+    p->tile_bytes = (size_t)PKV_BLOCK_SIZE * p->row_bytes;
+    p->layer_bytes = (size_t)d->num_blocks * d->num_kv_heads * p->tile_bytes;
+    p->layer_scales = is_quantized(d->kv_dtype) ? (size_t)d->num_blocks * d->num_kv_heads : 0;
+    const int L = d->num_layers;
+    try {
+        p->k_base.resize(L);
+        p->v_base.resize(L);
+        p->ks_base.assign(L, nullptr);
+        p->vs_base.assign(L, nullptr);
+    } catch (...) {
+        delete p;
+        return nullptr;
+    }
+    for (int l = 0; l < L; ++l) {
+        p->k_base[l] = static_cast<uint8_t*>(k[l]);
+        p->v_base[l] = static_cast<uint8_t*>(v[l]);
+        if (p->layer_scales) {
+            p->ks_base[l] = ks[l];
+            p->vs_base[l] = vs[l];
+        }
+    }
+    return p;
+}
+
 int kv_pool_create(const pkv_pool_desc* d, pkv_pool_t* out)
 {
     if (!out) return PKV_ERR_NULL;
@@ -168,13 +209,51 @@ int kv_pool_create(const pkv_pool_desc* d, pkv_pool_t* out)
     if (!d->k_data || !d->v_data) return PKV_ERR_NULL;
     if (is_quantized(d->kv_dtype) && (!d->k_scale || !d->v_scale)) return PKV_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(d->k_data) | reinterpret_cast<uintptr_t>(d->v_data)) & 15) return PKV_ERR_ARG;
-    pkv_pool* p = new (std::nothrow) pkv_pool();
+    // a dense pool: layer l starts l whole layers into each allocation
+    const size_t lb = (size_t)d->num_blocks * d->num_kv_heads * PKV_BLOCK_SIZE * row_bytes_of(d->kv_dtype, d->head_dim);
+    const size_t ls = (size_t)d->num_blocks * d->num_kv_heads;
+    void* k[PKV_MAX_LAYERS];
+    void* v[PKV_MAX_LAYERS];
+    float* ks[PKV_MAX_LAYERS];
+    float* vs[PKV_MAX_LAYERS];
+    for (int l = 0; l < d->num_layers; ++l) {
+        k[l] = static_cast<uint8_t*>(d->k_data) + (size_t)l * lb;
+        v[l] = static_cast<uint8_t*>(d->v_data) + (size_t)l * lb;
+        ks[l] = d->k_scale ? d->k_scale + (size_t)l * ls : nullptr;
+        vs[l] = d->v_scale ? d->v_scale + (size_t)l * ls : nullptr;
+    }
+    pkv_pool* p = new_pool(d, k, v, ks, vs);
     if (!p) return PKV_ERR_ARG;
-    p->d = *d;
-    p->row_bytes = row_bytes_of(d->kv_dtype, d->head_dim);
-    p->tile_bytes = (size_t)PKV_BLOCK_SIZE * p->row_bytes;
-    p->layer_bytes = (size_t)d->num_blocks * d->num_kv_heads * p->tile_bytes;
-    p->layer_scales = is_quantized(d->kv_dtype) ? (size_t)d->num_blocks * d->num_kv_heads : 0;
+    *out = p;
+    return PKV_OK;
+}
+
+int kv_pool_create_layers(const pkv_pool_desc* d, void* const* k_layers, void* const* v_layers,
+                          float* const* k_scale_layers, float* const* v_scale_layers, pkv_pool_t* out)
+{
+    if (!out) return PKV_ERR_NULL;
+    *out = nullptr;
+    int rc = validate_desc(d);
+    if (rc != PKV_OK) return rc;
+    if (!k_layers || !v_layers) return PKV_ERR_NULL;
+    const bool quant = is_quantized(d->kv_dtype);
+    if (quant && (!k_scale_layers || !v_scale_layers)) return PKV_ERR_NULL;
+    for (int l = 0; l < d->num_layers; ++l) {
+        if (!k_layers[l] || !v_layers[l]) return PKV_ERR_NULL;
+        if ((reinterpret_cast<uintptr_t>(k_layers[l]) | reinterpret_cast<uintptr_t>(v_layers[l])) & 15)
+            return PKV_ERR_ARG;
+        if (quant) {
+            if (!k_scale_layers[l] || !v_scale_layers[l]) return PKV_ERR_NULL;
+            if ((reinterpret_cast<uintptr_t>(k_scale_layers[l]) | reinterpret_cast<uintptr_t>(v_scale_layers[l])) & 3)
+                return PKV_ERR_ARG;
+        }
+    }
+    pkv_pool* p = new_pool(d, k_layers, v_layers, k_scale_layers, v_scale_layers);
+    if (!p) return PKV_ERR_ARG;
+    p->d.k_data = p->k_base[0];   // the first layer's, for callers that read the description back
+    p->d.v_data = p->v_base[0];
+    p->d.k_scale = p->ks_base[0];
+    p->d.v_scale = p->vs_base[0];
     *out = p;
     return PKV_OK;
 }
@@ -219,10 +298,10 @@ int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, int src_
     a.H_kv = d.num_kv_heads;
     a.d = d.head_dim;
     a.kv_dtype = d.kv_dtype;
-    a.k_pool = static_cast<uint8_t*>(d.k_data) + (size_t)layer * pool->layer_bytes;
-    a.v_pool = static_cast<uint8_t*>(d.v_data) + (size_t)layer * pool->layer_bytes;
-    a.k_scale = d.k_scale ? d.k_scale + (size_t)layer * pool->layer_scales : nullptr;
-    a.v_scale = d.v_scale ? d.v_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.k_pool = pool->k_base[layer];
+    a.v_pool = pool->v_base[layer];
+    a.k_scale = pool->ks_base[layer];
+    a.v_scale = pool->vs_base[layer];
     a.workspace = workspace;
     a.status = d.device_status;
     return launch_append(a, static_cast<cudaStream_t>(stream));
@@ -249,14 +328,22 @@ static int decode_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, i
     return PKV_OK;
 }
 
+// Split-K workspace: partials o [B][H_q][parts][d] and (m, l) [B][H_q][parts][2] (fp32), then
+// one int counter per (sequence, CTA of a partition) for the fused merge.
+static size_t decode_ws_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int parts)
+{
+    if (parts <= 1) return 0;
+    return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float) +
+           (size_t)num_seqs * ctas_per_partition(pool, num_q_heads) * sizeof(int);
+}
+
 size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_context_len,
                                     const pkv_decode_opts* opts)
 {
     if (!pool || num_seqs < 0 || num_q_heads <= 0 || max_context_len < 0) return 0;
     int P, parts;
     if (decode_partitioning(pool, num_seqs, num_q_heads, max_context_len, opts, &P, &parts) != PKV_OK) return 0;
-    if (parts <= 1) return 0;
-    return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float);
+    return decode_ws_bytes(pool, num_seqs, num_q_heads, parts);
 }
 
 int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, const int32_t* block_tables,
@@ -283,7 +370,7 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     int P, parts;
     int rc = decode_partitioning(pool, num_seqs, num_q_heads, max_context_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;
-    const size_t need = parts > 1 ? (size_t)num_seqs * num_q_heads * parts * (d.head_dim + 2) * sizeof(float) : 0;
+    const size_t need = decode_ws_bytes(pool, num_seqs, num_q_heads, parts);
     if (need && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 15)))
         return PKV_ERR_WORKSPACE;
     const CUtensorMap *tmk = nullptr, *tmv = nullptr;
@@ -306,12 +393,15 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     a.part_tokens = P;
     a.max_parts = parts;
     a.scale = scale;
-    a.k_scale = d.k_scale ? d.k_scale + (size_t)layer * pool->layer_scales : nullptr;
-    a.v_scale = d.v_scale ? d.v_scale + (size_t)layer * pool->layer_scales : nullptr;
+    a.k_scale = pool->ks_base[layer];
+    a.v_scale = pool->vs_base[layer];
     a.out = out;
     float* ws = static_cast<float*>(workspace);
     a.ws_o = need ? ws : nullptr;
     a.ws_ml = need ? ws + (size_t)num_seqs * num_q_heads * parts * d.head_dim : nullptr;
+    a.counters = need ? reinterpret_cast<int*>(ws + (size_t)num_seqs * num_q_heads * parts * (d.head_dim + 2))
+                      : nullptr;
+    a.counter_count = need ? num_seqs * ctas_per_partition(pool, num_q_heads) : 0;
     a.status = d.device_status;
     a.engine = engine;
     a.window = opts ? opts->sliding_window : 0;
@@ -518,6 +608,24 @@ int paged_prefill_chunk_attn_window(pkv_pool_t pool, int layer, const void* q, i
         return launch_prefill_tc(a, &tmq, tmk, tmv, static_cast<cudaStream_t>(stream));
     }
     return launch_prefill(a, tmk, tmv, static_cast<cudaStream_t>(stream));
+}
+
+int pkv_test_withhold_copy(int tile, long long wait_cycles)
+{
+    if (tile < 0) {
+        g_hold_tile.store(-1);
+        g_wait_cycles.store(kDefaultWaitCycles);
+        return PKV_OK;
+    }
+    if (wait_cycles <= 0 || wait_cycles > kDefaultWaitCycles) return PKV_ERR_ARG;
+    g_wait_cycles.store(wait_cycles);
+    g_hold_tile.store(tile);
+    return PKV_OK;
+}
+
+int pkv_get_device_status(pkv_pool_t pool, void* stream, int32_t* status_out)
+{
+    return pkv_read_device_status(pool, stream, status_out);
 }
 
 int pkv_read_device_status(pkv_pool_t pool, void* stream, int32_t* status_out)

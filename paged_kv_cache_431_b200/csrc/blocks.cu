@@ -7,9 +7,12 @@
 // preemption": a preempted sequence's blocks are swapped to host memory and back.
 //
 // A block is, for every layer, its H_kv tiles of K and of V (H_kv * 16 * row_bytes bytes
-// each) and, for quantized pools, its 2 * H_kv scales.  All moves are 16-byte vector
-// copies, one thread per 16 bytes, bound by HBM (copies) or by the host link (swaps:
-// the kernels read / write pinned host memory directly through its device mapping).
+// each, contiguous) and, for quantized pools, its 2 * H_kv scales.  Layers may live in
+// separate allocations: the kernels get every layer's base pointers as a parameter.  All
+// moves are 16-byte vector copies.  A copy runs one CTA per (pair, layer, K/V) span with
+// several loads in flight per thread, bound by HBM; a swap runs one thread per 16 bytes
+// over the host link (the kernel reads / writes pinned host memory directly through its
+// device mapping).
 #include "common.cuh"
 #include "internal.h"
 
@@ -19,10 +22,16 @@ namespace {
 
 struct BlockGeom {
     size_t tile_row;      // bytes of one block's K (or V) in one layer: H_kv * 16 * row_bytes
-    size_t layer_bytes;   // bytes of one layer's K (or V) pool
     size_t scales;        // scales per block per layer per K/V (H_kv), 0 for 16-bit pools
-    size_t layer_scales;  // scales per layer (N * H_kv)
     int L, N;
+};
+
+// Every layer's K / V pool and K / V scales (scales null for 16-bit pools), passed by value.
+struct LayerBases {
+    uint8_t* k[PKV_MAX_LAYERS];
+    uint8_t* v[PKV_MAX_LAYERS];
+    float* ks[PKV_MAX_LAYERS];
+    float* vs[PKV_MAX_LAYERS];
 };
 
 // Host layout of one swapped block: [L][K, V][tile_row bytes], then [L][K, V][scales] fp32.
@@ -38,7 +47,7 @@ constexpr int kCopyThreads = 256;
 constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(kCopyThreads)
-copy_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g, const int32_t* __restrict__ src,
+copy_blocks_kernel(const __grid_constant__ LayerBases lb, BlockGeom g, const int32_t* __restrict__ src,
                    const int32_t* __restrict__ dst, int32_t* status)
 {
     const int item = blockIdx.x;                 // (pair * L + layer) * 2 + is_v
@@ -50,7 +59,7 @@ copy_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g, co
         if (threadIdx.x == 0 && layer == 0 && !is_v) flag_status(status, PKV_DEV_BAD_BLOCK);
         return;
     }
-    uint8_t* base = (is_v ? v : k) + (size_t)layer * g.layer_bytes;
+    uint8_t* base = is_v ? lb.v[layer] : lb.k[layer];
     const uint4* from = reinterpret_cast<const uint4*>(base + (size_t)sb * g.tile_row);
     uint4* to = reinterpret_cast<uint4*>(base + (size_t)db * g.tile_row);
     const int chunks = (int)(g.tile_row / 16);
@@ -68,13 +77,13 @@ copy_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g, co
         }
     }
     if (g.scales) {
-        float* sc = (is_v ? vs : ks) + (size_t)layer * g.layer_scales;
+        float* sc = is_v ? lb.vs[layer] : lb.ks[layer];
         for (size_t h = threadIdx.x; h < g.scales; h += kCopyThreads) sc[(size_t)db * g.scales + h] = sc[(size_t)sb * g.scales + h];
     }
 }
 
 // Swap out (to_host) or in: block blocks[j] <-> host slot j.
-__global__ void swap_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs, BlockGeom g,
+__global__ void swap_blocks_kernel(const __grid_constant__ LayerBases lb, BlockGeom g,
                                    const int32_t* __restrict__ blocks, int n, uint8_t* host, bool to_host,
                                    int32_t* status)
 {
@@ -94,12 +103,12 @@ __global__ void swap_blocks_kernel(uint8_t* k, uint8_t* v, float* ks, float* vs,
         return;
     }
     uint8_t* hb = host + (size_t)j * swap_block_bytes(g);
-    uint4* dev = reinterpret_cast<uint4*>((is_v ? v : k) + (size_t)layer * g.layer_bytes + (size_t)blk * g.tile_row) + c;
+    uint4* dev = reinterpret_cast<uint4*>((is_v ? lb.v[layer] : lb.k[layer]) + (size_t)blk * g.tile_row) + c;
     uint4* hst = reinterpret_cast<uint4*>(hb + ((size_t)layer * 2 + (is_v ? 1 : 0)) * g.tile_row) + c;
     if (to_host) *hst = *dev;
     else *dev = *hst;
     if (g.scales && c < g.scales) {
-        float* sc = (is_v ? vs : ks) + (size_t)layer * g.layer_scales + (size_t)blk * g.scales + c;
+        float* sc = (is_v ? lb.vs[layer] : lb.ks[layer]) + (size_t)blk * g.scales + c;
         float* hs = reinterpret_cast<float*>(hb + (size_t)g.L * 2 * g.tile_row) + ((size_t)layer * 2 + (is_v ? 1 : 0)) * g.scales + c;
         if (to_host) *hs = *sc;
         else *sc = *hs;
@@ -110,9 +119,7 @@ BlockGeom geom_of(const pkv_pool* pool)
 {
     BlockGeom g;
     g.tile_row = (size_t)pool->d.num_kv_heads * pool->tile_bytes;
-    g.layer_bytes = pool->layer_bytes;
     g.scales = pool->layer_scales ? (size_t)pool->d.num_kv_heads : 0;
-    g.layer_scales = pool->layer_scales;
     g.L = pool->d.num_layers;
     g.N = pool->d.num_blocks;
     return g;
@@ -126,16 +133,19 @@ static int launch_moves(bool copy, const pkv_pool* pool, const int32_t* a, const
     const int threads = 256;
     const size_t grid = (total + threads - 1) / threads;
     if (grid > 0x7fffffffULL) return PKV_ERR_ARG;
-    uint8_t* k = static_cast<uint8_t*>(pool->d.k_data);
-    uint8_t* v = static_cast<uint8_t*>(pool->d.v_data);
+    LayerBases lb = {};
+    for (int l = 0; l < g.L; ++l) {
+        lb.k[l] = pool->k_base[l];
+        lb.v[l] = pool->v_base[l];
+        lb.ks[l] = pool->ks_base[l];
+        lb.vs[l] = pool->vs_base[l];
+    }
     if (copy) {
         const size_t items = (size_t)n * g.L * 2;
         if (items > 0x7fffffffULL) return PKV_ERR_ARG;
-        copy_blocks_kernel<<<(unsigned)items, kCopyThreads, 0, s>>>(k, v, pool->d.k_scale, pool->d.v_scale, g, a, b,
-                                                                    pool->d.device_status);
+        copy_blocks_kernel<<<(unsigned)items, kCopyThreads, 0, s>>>(lb, g, a, b, pool->d.device_status);
     } else
-        swap_blocks_kernel<<<(unsigned)grid, threads, 0, s>>>(k, v, pool->d.k_scale, pool->d.v_scale, g, a, n, host,
-                                                              to_host, pool->d.device_status);
+        swap_blocks_kernel<<<(unsigned)grid, threads, 0, s>>>(lb, g, a, n, host, to_host, pool->d.device_status);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

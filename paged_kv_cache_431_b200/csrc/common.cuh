@@ -17,8 +17,10 @@ namespace pkv {
 
 constexpr int kBlock = PKV_BLOCK_SIZE;
 
-// Upper bound on one wait for a bulk copy: about 1 s at the B200's clock.  A copy that
-// has not landed by then will never land; the kernel records PKV_DEV_TIMEOUT and stops.
+// Default upper bound on one wait for a bulk copy: about 1 s at the B200's clock.  A copy
+// that has not landed by then will never land; the kernel records PKV_DEV_TIMEOUT and stops.
+// The kernels take the bound from their launch (pkv_test_withhold_copy lowers it for a test
+// of that path).
 constexpr long long kWaitCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
@@ -66,13 +68,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for phase `parity` of the barrier to complete, giving up after kWaitCycles.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+// Wait for phase `parity` of the barrier to complete, giving up after `limit` SM cycles.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, long long limit = kWaitCycles)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles) return false;
+        if (clock64() - t0 > limit) return false;
     }
     return true;
 }

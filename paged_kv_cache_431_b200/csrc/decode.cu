@@ -28,9 +28,11 @@
 //     shuffles.  Masked (past-the-end) tokens get -inf scores and zeroed V, so stale or
 //     poisoned slots never reach the result.
 //   * Split-K: a sequence longer than one partition writes per-partition (o, m, l)
-//     partials; decode_reduce merges them with the log-sum-exp rule.  The shared-prefix
-//     (cascade) form starts the partitions after the prefix and merges them with the
-//     prefix's partials written by the tensor-core prefill kernel.
+//     partials and counts itself done on a per-(sequence, head group) counter; the CTA that
+//     completes the count merges them with the log-sum-exp rule (no second launch).  The
+//     shared-prefix (cascade) form starts the partitions after the prefix and leaves the
+//     merge, with the prefix's partials written by the tensor-core prefill kernel, to
+//     decode_reduce.
 #include "decode_common.cuh"
 
 namespace pkv {
@@ -115,6 +117,7 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         const int row = (tbl[j] * p.H_kv + g) * kBlock;
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        if (j == p.hold_tile) return;   // test hook: the stage's bytes never arrive
 #pragma unroll
         for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + x * 2048, &tmK, x * 64, row, bar);
 #pragma unroll
@@ -153,7 +156,8 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
     bool ok = true;
     for (; j < ntiles; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1)) {
+        // the whole warp gives up together (its mma.sync needs every lane)
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1, p.wait_cycles))) {
             ok = false;
             break;
         }
@@ -270,25 +274,31 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 fence_proxy_async_smem();
                 mbar_arrive(smem_u32(&empty[s]));
             }
+            bool refilled = true;
             if (threadIdx.x == 0 && j + STAGES < ntiles) {
-                if (mbar_wait_bounded(smem_u32(&empty[s]), (j / STAGES) & 1)) {
-                    issue(j + STAGES);
-                } else {
-                    ok = false;
-                    ++j;
-                    break;
-                }
+                refilled = mbar_wait_bounded(smem_u32(&empty[s]), (j / STAGES) & 1, p.wait_cycles);
+                if (refilled) issue(j + STAGES);
+            }
+            if (!__shfl_sync(0xffffffffu, refilled ? 1 : 0, 0)) {   // warp 0 stops; the others time out
+                ok = false;
+                ++j;
+                break;
             }
         }
     }
 
-    if (!ok) {
+    if (!ok) {   // no copy may still be landing in this CTA's shared memory when it exits
         if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
         for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
-            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
+            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1, p.wait_cycles);
     }
-    if constexpr (NW > 1) __syncthreads();   // every warp is done with the ring before the staging reuses it
-    if (!ok) return;
+    if constexpr (NW > 1) {
+        // every warp is done with the ring before the staging reuses it; a warp that gave up
+        // stops the whole CTA (the epilogue's barriers need every warp)
+        if (__syncthreads_or(!ok)) return;
+    } else {
+        if (!ok) return;
+    }
 
     // ---- epilogue: O rows [head][dim] through shared memory, then coalesced stores
 #pragma unroll
@@ -338,6 +348,10 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                     *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) = ml;
                 }
             }
+        }
+        if (p.counters) {   // the CTA that completes this (sequence, head group) merges all partitions
+            __shared__ int s_last;
+            if (last_partition(p, b, nparts, &s_last)) merge_partials<D>(p, row0, GC, nparts, lane);
         }
     }
 }
@@ -452,6 +466,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.out = a.out;
     p.ws_o = a.ws_o;
     p.ws_ml = a.ws_ml;
+    p.counters = nullptr;
     p.status = a.status;
     p.W = a.W;
     p.H_q = a.H_q;
@@ -468,9 +483,21 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.hgroups = (a.G + 15) / 16;
     p.q_bf16 = a.q_dtype == PKV_BF16;
     p.scale_log2 = a.scale * kLog2e;
+    const WaitHook hook = wait_hook();
+    p.hold_tile = hook.hold_tile;
+    p.wait_cycles = hook.wait_cycles;
 
     const dim3 grid(a.max_parts, a.H_kv * p.hgroups, a.B);
     const int nht = a.G <= 8 ? 1 : 2;   // 8 or 16 query heads per CTA
+    // The tensor-core engines merge the split-K partials in the CTA that finishes a
+    // (sequence, head group) last; its counters start at zero (one small memset per call: the
+    // workspace is the caller's and may hold anything).  The CUDA-core engines and the cascade
+    // form merge in decode_reduce.
+    if (a.counters && a.max_parts > 1 && a.part_base == 0 && a.engine == 1) {
+        if (cudaMemsetAsync(a.counters, 0, (size_t)a.counter_count * sizeof(int), s) != cudaSuccess)
+            return PKV_ERR_CUDA;
+        p.counters = a.counters;
+    }
     int rc = PKV_ERR_UNSUPPORTED;
     if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && (a.engine == 2 || a.engine == 3)) {
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
@@ -488,7 +515,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         rc = launch_decode_quant(p, a.kv_dtype, a.d, nht, grid, s, tmk, tmv);
     }
     if (rc != PKV_OK) return rc;
-    if (a.max_parts > 1 || a.part_base > 0) {
+    if ((a.max_parts > 1 && !p.counters) || a.part_base > 0) {
         // programmatic dependent launch: scheduled while the decode grid's last wave runs
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(a.H_q, a.B);

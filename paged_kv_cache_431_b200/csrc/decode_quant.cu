@@ -9,7 +9,9 @@
 // TMA ring of K/V code tiles, online softmax, split-K partials), with dequantization
 // fused into the fragment loads:
 //   * codes are converted to fp16 in registers and fed to mma.sync m16n8k16 (f16 in,
-//     fp32 accumulate); q is converted to fp16 once per warp:
+//     fp32 accumulate); q is scaled by a power of two chosen per CTA (its largest |q|
+//     brought near 2^14, exact, undone in the score) and converted to fp16 once per warp,
+//     so a bf16 q keeps its range:
 //       - integer K codes: the code plus its offset (c + 128, c + 8) is moved into the
 //         significand of an fp16 subnormal (one byte permute or one logic op per pair,
 //         exact); the offset's share of every score, offset * sum(q), is subtracted once
@@ -107,11 +109,13 @@ __device__ __forceinline__ float pow2f(int e)
     return __int_as_float((127 + e) << 23);
 }
 
-// Shift e in [-60, 60] that brings x > 0 into [2^13, 2^14) as x * 2^e (60 for x = 0).
+// Shift e in [-100, 100] that brings x > 0 into [2^13, 2^14) as x * 2^e (100 for x = 0 or a
+// subnormal x).  The bound keeps 2^e, 2^-e and 2^(24 - e) finite floats; it covers every
+// |q| below 2^114.
 __device__ __forceinline__ int pow2_shift(float x)
 {
     const int ex = (int)((__float_as_uint(x) >> 23) & 0xffu) - 127;   // x in [2^ex, 2^(ex+1)) if normal
-    return max(-60, min(60, 13 - ex));
+    return max(-100, min(100, 13 - ex));
 }
 
 __device__ __forceinline__ float warp_max(float v)
@@ -250,9 +254,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     constexpr int ROW = Cfg::ROW, SWZ = Cfg::SWZ;
     // integer K codes enter Q . K^T as subnormals u * 2^-24 with u = c + OFF; odd int4
     // nibbles enter as 16 u, and their q is pre-divided by 16.  q is pre-scaled by a power
-    // of two chosen per CTA (largest |q| brought near 2^14) so that the products stay well
-    // clear of the bottom of the accumulator's range; the scaling is exact and is undone,
-    // with the offset, in the score.
+    // of two chosen per CTA (largest |q| brought near 2^14): for integer codes the products
+    // then stay well clear of the bottom of the accumulator's range, and for every dtype a
+    // bf16 q of any magnitude up to 2^113 fits fp16 (a bf16 q above 65504 would otherwise
+    // become inf).  The scaling is exact and is undone, with the offset, in the score.
     constexpr bool SUBN = DT != PKV_FP8E4M3;
     constexpr float OFF = DT == PKV_INT8 ? 128.f : 8.f;
     constexpr float ODD = DT == PKV_INT4 ? 0.0625f : 1.f;   // q factor on k-slots 8..15
@@ -311,6 +316,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         const int row = (tbl[j] * p.H_kv + g) * kBlock;
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        if (j == p.hold_tile) return;   // test hook: the stage's bytes never arrive
         tma_load_2d(kdst, &tmK, 0, row, bar);
         tma_load_2d(kdst + Cfg::TILE, &tmV, 0, row, bar);
     };
@@ -323,7 +329,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     // per head row r, r + 8: the part of 2^24 * (q . k) that the code offset adds
     uint32_t qa[Cfg::KS][4];
     float qoff[2] = {0.f, 0.f};
-    int eq = 0;   // q is multiplied by 2^eq (integer codes), which brings max |q| to [2^13, 2^14)
+    int eq = 0;   // q is multiplied by 2^eq, which brings max |q| to [2^13, 2^14)
     {
         const bool bf = p.q_bf16;
         const uint16_t* qh = static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D;
@@ -332,14 +338,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             return bf ? __uint_as_float((uint32_t)u << 16) : __half2float(__ushort_as_half(u));
         };
         const bool r0 = r < GC, r1 = (NHT == 2) && (r + 8 < GC);
-        float qs = 1.f, qo = ODD;
-        if constexpr (SUBN) {
-            float qmax = 0.f;
-            for (int i = lane; i < GC * D; i += 32) qmax = fmaxf(qmax, fabsf(qv(0, i)));
-            eq = pow2_shift(warp_max(qmax));
-            qs = pow2f(eq);
-            qo = qs * ODD;
-        }
+        float qmax = 0.f;
+        for (int i = lane; i < GC * D; i += 32) qmax = fmaxf(qmax, fabsf(qv(0, i)));
+        eq = pow2_shift(warp_max(qmax));
+        const float qs = pow2f(eq), qo = qs * ODD;
 #pragma unroll
         for (int ks = 0; ks < Cfg::KS; ++ks) {
             const int d0 = kdim<DT, D>(ks, qd, 0), d1 = kdim<DT, D>(ks, qd, 1);
@@ -363,7 +365,8 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             }
         }
     }
-    const float kq = pow2f(24 - eq);     // log2-domain score = (acc * 2^(24-eq) + qoff) * sl
+    // log2-domain score = (acc * 2^(24-eq) + qoff) * sl for integer codes, acc * 2^-eq * sl for fp8
+    const float kq = pow2f(SUBN ? 24 - eq : -eq);
 
     float o[Cfg::MT][NHT][4];
 #pragma unroll
@@ -378,7 +381,8 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     bool ok = true;
     for (; j < ntiles; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1)) {
+        // the whole warp gives up together (its mma.sync needs every lane)
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1, p.wait_cycles))) {
             ok = false;
             break;
         }
@@ -409,7 +413,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         }
 
         const float sl = p.scale_log2 * sc_kv.x;
-        const float slk = SUBN ? sl * kq : sl;
+        const float slk = sl * kq;
         float pr[2][4];
         float alpha[2];
 #pragma unroll
@@ -518,10 +522,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         }
     }
 
-    if (!ok) {
+    if (!ok) {   // no copy may still be landing in this CTA's shared memory when it exits
         if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
         for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
-            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
+            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1, p.wait_cycles);
         return;
     }
 
@@ -568,6 +572,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
                 *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) =
                     make_float2(m_run[hr], l_run[hr]);
         }
+    }
+    if (!final_out && p.counters) {   // the CTA that completes this (sequence, head group) merges
+        __shared__ int s_last;
+        if (last_partition(p, b, nparts, &s_last)) merge_partials<D>(p, row0, GC, nparts, lane);
     }
 }
 

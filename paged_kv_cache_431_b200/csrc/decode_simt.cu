@@ -110,6 +110,7 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         const int row = (tbl[j] * p.H_kv + g) * kBlock;
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        if (j == p.hold_tile) return;   // test hook: the stage's bytes never arrive
 #pragma unroll
         for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + x * 2048, &tmK, x * 64, row, bar);
 #pragma unroll
@@ -142,7 +143,8 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     bool ok = true;
     for (; j < ntiles; ++j) {
         const int s = j % STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1)) {
+        // the whole warp gives up together (its shuffles need every lane)
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1, p.wait_cycles))) {
             ok = false;
             break;
         }
@@ -256,10 +258,10 @@ decode_simt_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             issue(j + STAGES);
         }
     }
-    if (!ok) {
+    if (!ok) {   // no copy may still be landing in this CTA's shared memory when it exits
         if (lane == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
         for (int jj = j; jj < min(ntiles, j + STAGES); ++jj)
-            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1);
+            mbar_wait_bounded(smem_u32(&bars[jj % STAGES]), (jj / STAGES) & 1, p.wait_cycles);
         return;
     }
 

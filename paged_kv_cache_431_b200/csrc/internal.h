@@ -16,12 +16,25 @@ struct pkv_pool {
     size_t tile_bytes;         // 16 rows: one (block, kv head) tile
     size_t layer_bytes;        // bytes of one layer's K (or V) pool
     size_t layer_scales;       // fp32 scales per layer (N * H_kv), 0 for 16-bit pools
+    // Per layer: base of its K and V pools and of its K and V scales (null for 16-bit pools).
+    // Dense pools: offsets into desc.k_data etc.; kv_pool_create_layers: the caller's pointers.
+    std::vector<uint8_t*> k_base, v_base;
+    std::vector<float*> ks_base, vs_base;
     std::mutex mu;             // guards the lazily built tensor maps
     bool maps_ready = false;
     std::vector<CUtensorMap> tmk, tmv;   // per layer: K and V pool as a 2-D tensor
 };
 
 namespace pkv {
+
+// The test hook of pkv_test_withhold_copy, read by every attention launcher: the CTA-local
+// index of the K/V tile whose copy is withheld (-1: none) and the wait bound in SM cycles.
+struct WaitHook {
+    int hold_tile;
+    long long wait_cycles;
+};
+WaitHook wait_hook();
+constexpr long long kDefaultWaitCycles = 2000000000LL;   // about 1 s at the B200's clock
 
 int row_bytes_of(int dtype, int head_dim);
 bool is_quantized(int dtype);
@@ -46,6 +59,8 @@ struct DecodeArgs {
     float* out;
     float* ws_o;            // [B][H_q][max_parts][d]
     float* ws_ml;           // [B][H_q][max_parts][2]
+    int* counters = nullptr;    // fused split-K merge: counter_count ints after the partials
+    int counter_count = 0;
     int32_t* status;
     int engine;             // 1 mma, 2 fma
     int tok_base = 0;       // first token the partitions cover (cascade: the prefix length)

@@ -16,6 +16,8 @@
 // shapes the tcgen05 form (prefill_tc.cu) does not: head dim 64, group sizes that do not
 // divide 128, and sliding-window chunks (a row at position p sees p - window + 1 .. p;
 // key tiles and blocks before every window of the CTA are not read).
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -46,6 +48,8 @@ struct PrefillParams {
     int W, P0, C, H_q, H_kv, G, N;
     int window;             // sliding window (keys a row sees, itself included); 0 = all earlier
     float scale_log2;
+    int hold_tile;          // test hook: this CTA-local tile's copy is never issued (-1: none)
+    long long wait_cycles;  // bound of every wait on a copy (SM cycles)
 };
 
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int t, int c)
@@ -61,7 +65,7 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     using Cfg = PrefillCfg<D>;
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[Cfg::STAGES];
-    __shared__ int s_fail;
+    __shared__ int s_fail_t;   // the first key tile whose copy a thread gave up on (INT_MAX: none)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.y;
@@ -81,7 +85,7 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     if (tid == 0) {
-        s_fail = 0;
+        s_fail_t = INT_MAX;
         for (int s = 0; s < Cfg::STAGES; ++s) mbar_init(smem_u32(&bars[s]), 1);
         mbar_fence_init();
         prefetch_tensormap(&tmK);
@@ -94,6 +98,7 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
         const uint32_t bar = smem_u32(&bars[s]);
         const uint32_t kdst = smem_u32(smem + s * Cfg::STAGE);
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
+        if (t - t_begin == p.hold_tile) return;   // test hook: the stage's bytes never arrive
         // all four table entries first, so their loads overlap
         int rows[4];
 #pragma unroll
@@ -157,9 +162,11 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
     const int kwin_lo = p.window > 0 ? max(0, kmin_warp - p.window) : 0;
     const int kwin_hi = p.window > 0 ? max(0, p.P0 + min(p.C - 1, (row_cta + warp * 16 + 15) / p.G) + 1 - p.window) : 0;
 
+    int t_stop = ntiles;   // the tile the CTA stopped at (ntiles: it did not)
     for (int t = t_begin; t < ntiles; ++t) {
         const int s = (t - t_begin) % Cfg::STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), ((t - t_begin) / Cfg::STAGES) & 1)) atomicExch(&s_fail, 1);
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), ((t - t_begin) / Cfg::STAGES) & 1, p.wait_cycles))
+            atomicMin(&s_fail_t, t);   // this tile's data is not there: computed on, but never written out
         const uint32_t kb = smem_u32(smem + s * Cfg::STAGE);
         const uint32_t vb = kb + Cfg::KBYTES;
         const int key0 = t * kKeys;
@@ -263,13 +270,24 @@ prefill_mma_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm
             }
         }
         __syncthreads();
+        // A give-up in this tile was recorded before the barrier; one in a later tile records a
+        // larger index, so every thread takes the same decision here.
+        if (s_fail_t <= t) {
+            t_stop = t;
+            break;
+        }
         if (tid == 0 && t + Cfg::STAGES < ntiles) {
             fence_proxy_async_smem();
             issue(t + Cfg::STAGES);
         }
     }
-    if (s_fail) {
-        if (tid == 0) flag_status(p.status, PKV_DEV_TIMEOUT);
+    if (t_stop < ntiles) {   // no copy may still be landing in this CTA's shared memory when it exits
+        if (tid == 0) {
+            flag_status(p.status, PKV_DEV_TIMEOUT);
+            for (int t = t_stop; t < min(ntiles, t_stop + Cfg::STAGES); ++t)
+                mbar_wait_bounded(smem_u32(&bars[(t - t_begin) % Cfg::STAGES]), ((t - t_begin) / Cfg::STAGES) & 1,
+                                  p.wait_cycles);
+        }
         return;
     }
 #pragma unroll
@@ -317,6 +335,9 @@ int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorM
     p.N = a.N;
     p.scale_log2 = a.scale * kLog2e;
     p.window = a.window;
+    const WaitHook hook = wait_hook();
+    p.hold_tile = hook.hold_tile;
+    p.wait_cycles = hook.wait_cycles;
     const bool bf = a.kv_dtype == PKV_BF16;
     if (a.d == 128) return bf ? launch_prefill_mma<128, true>(p, s, tmk, tmv) : launch_prefill_mma<128, false>(p, s, tmk, tmv);
     if (a.d == 64) return bf ? launch_prefill_mma<64, true>(p, s, tmk, tmv) : launch_prefill_mma<64, false>(p, s, tmk, tmv);

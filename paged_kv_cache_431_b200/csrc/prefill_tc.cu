@@ -59,6 +59,8 @@ struct TcParams {
     int cascade, nkeys, slots;
     float* ws_o;
     float* ws_ml;
+    int hold_tile;          // test hook: the K copy of this CTA-local key tile is never issued (-1: none)
+    long long wait_cycles;  // bound of every wait (SM cycles)
 };
 
 // ---- tcgen05 wrappers ------------------------------------------------------
@@ -172,10 +174,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 
 // Wait with a bound; on timeout record it and raise the CTA's abort flag.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status)
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                                              long long limit)
 {
     if (*abort_flag) return false;
-    if (mbar_wait_bounded(bar, parity)) return true;
+    if (mbar_wait_bounded(bar, parity, limit)) return true;
     *abort_flag = 1;
     flag_status(status, PKV_DEV_TIMEOUT);
     return false;
@@ -212,6 +215,7 @@ struct Bars {
     uint64_t s_full[kQT];      // S(x, t) is in TMEM (every earlier MMA of the CTA is done too)
     uint64_t p_full[kQT];      // P(x, t) stored by the four softmax warps of tile x
     uint64_t o_done[kQT];      // the last P . V of tile x is done
+    uint64_t mma_drain;        // every MMA the issuer launched is done (before TMEM is freed)
 };
 
 template <bool BF16>
@@ -256,6 +260,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             mbar_init(smem_u32(&bars.p_full[x]), 4);
             mbar_init(smem_u32(&bars.o_done[x]), 1);
         }
+        mbar_init(smem_u32(&bars.mma_drain), 1);
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -315,20 +320,23 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             }
             bool go = true;
             if (lane == 0 && t >= kNS)
-                go = wait_or_abort(smem_u32(&bars.k_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
+                go = wait_or_abort(smem_u32(&bars.k_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status, p.wait_cycles);
             if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&bars.k_full[s]);
                 mbar_arrive_expect_tx(fb, kKVBytes);
+                if (t != p.hold_tile) {   // test hook: the withheld tile's K bytes never arrive
 #pragma unroll
-                for (int kb = 0; kb < kBlkPerTile; ++kb)
+                    for (int kb = 0; kb < kBlkPerTile; ++kb)
 #pragma unroll
-                    for (int x = 0; x < 2; ++x)
-                        tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, row_of[kb], fb);
+                        for (int x = 0; x < 2; ++x)
+                            tma_load_2d(sK + s * kKVBytes + x * (kKVBytes / 2) + kb * 2048, &tmK, 64 * x, row_of[kb],
+                                        fb);
+                }
             }
             issued_k = t + 1;
             if (lane == 0 && t >= kNS)
-                go = wait_or_abort(smem_u32(&bars.v_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status);
+                go = wait_or_abort(smem_u32(&bars.v_empty[s]), ((t - kNS) / kNS) & 1, &s_abort, p.status, p.wait_cycles);
             if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
             if (lane == 0) {
                 const uint32_t fb = smem_u32(&bars.v_full[s]);
@@ -344,10 +352,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         // do not leave while copies into this CTA's shared memory may be in flight
         if (lane == 0 && s_abort) {
             for (int t = max(0, issued_k - kNS); t < issued_k; ++t)
-                mbar_wait_bounded(smem_u32(&bars.k_full[t % kNS]), (t / kNS) & 1);
+                mbar_wait_bounded(smem_u32(&bars.k_full[t % kNS]), (t / kNS) & 1, p.wait_cycles);
             for (int t = max(0, issued - kNS); t < issued; ++t)
-                mbar_wait_bounded(smem_u32(&bars.v_full[t % kNS]), (t / kNS) & 1);
-            mbar_wait_bounded(qb, 0);
+                mbar_wait_bounded(smem_u32(&bars.v_full[t % kNS]), (t / kNS) & 1, p.wait_cycles);
+            mbar_wait_bounded(qb, 0, p.wait_cycles);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -375,8 +383,8 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                     umma_ts(tmem + 256 * x + 128, a + 16, bv, id_pv, true);
                 }
             };
-            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status) &&
-                      wait_or_abort(smem_u32(&bars.k_full[0]), 0, &s_abort, p.status);
+            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status, p.wait_cycles) &&
+                      wait_or_abort(smem_u32(&bars.k_full[0]), 0, &s_abort, p.status, p.wait_cycles);
             if (ok) {
                 tc_fence_after();
                 qk(0, 0);
@@ -389,12 +397,12 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 const int s = t % kNS, s1 = (t + 1) % kNS;
                 const bool more = t + 1 < ntiles;
                 // tile A: P . V, then its next scores
-                if (!wait_or_abort(smem_u32(&bars.p_full[0]), t & 1, &s_abort, p.status)) break;
-                if (!wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status)) break;
+                if (!wait_or_abort(smem_u32(&bars.p_full[0]), t & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
                 tc_fence_after();
                 pv(0, s, t == 0);
                 if (more) {
-                    if (!wait_or_abort(smem_u32(&bars.k_full[s1]), ((t + 1) / kNS) & 1, &s_abort, p.status)) break;
+                    if (!wait_or_abort(smem_u32(&bars.k_full[s1]), ((t + 1) / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
                     tc_fence_after();
                     qk(0, s1);
                     umma_commit(smem_u32(&bars.s_full[0]));
@@ -402,7 +410,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                     umma_commit(smem_u32(&bars.o_done[0]));
                 }
                 // tile B
-                if (!wait_or_abort(smem_u32(&bars.p_full[1]), t & 1, &s_abort, p.status)) break;
+                if (!wait_or_abort(smem_u32(&bars.p_full[1]), t & 1, &s_abort, p.status, p.wait_cycles)) break;
                 tc_fence_after();
                 pv(1, s, t == 0);
                 umma_commit(smem_u32(&bars.v_empty[s]));
@@ -414,6 +422,9 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                     umma_commit(smem_u32(&bars.o_done[1]));
                 }
             }
+            // Every MMA this thread issued, also on an abort, is done before TMEM is freed.
+            umma_commit(smem_u32(&bars.mma_drain));
+            mbar_wait_bounded(smem_u32(&bars.mma_drain), 0, p.wait_cycles);
         }
     } else {
         // ------------------------------------------------------------ softmax
@@ -434,7 +445,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         float m_used = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
-            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[x]), t & 1, &s_abort, p.status))) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[x]), t & 1, &s_abort, p.status, p.wait_cycles))) {
                 ok = false;
                 break;
             }
@@ -516,7 +527,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             // stale).  Tile A's warps do it before their P . V, which runs before tile B's.
             if (x == 0 && t == ntiles - 1 && key0 + kBN > seq_len) {   // only the last split's last tile
                 const int s = t % kNS;
-                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status))) {
+                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles))) {
                     ok = false;
                     break;
                 }
@@ -534,7 +545,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[x]));
         }
-        if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done[x]), 0, &s_abort, p.status))) {
+        if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done[x]), 0, &s_abort, p.status, p.wait_cycles))) {
             tc_fence_after();
             const bool valid = pos < p.C;
             const float inv = p.cascade ? 1.f : 1.f / l_run;
@@ -613,6 +624,9 @@ int launch_prefill_tc(const PrefillArgs& a, const CUtensorMap* tmq, const CUtens
     p.slots = a.ws_slots;
     p.ws_o = a.ws_o;
     p.ws_ml = a.ws_ml;
+    const WaitHook hook = wait_hook();
+    p.hold_tile = hook.hold_tile;
+    p.wait_cycles = hook.wait_cycles;
     auto kern = a.kv_dtype == PKV_BF16 ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
         return PKV_ERR_CUDA;

@@ -15,6 +15,7 @@ import torch
 from . import build as _build
 
 BLOCK_SIZE = 16
+MAX_LAYERS = 256          # PKV_MAX_LAYERS
 F16, BF16, INT8, INT4, FP8E4M3 = 0, 1, 2, 3, 4
 QUANTIZED = (INT8, INT4, FP8E4M3)
 DEV_BAD_BLOCK, DEV_BAD_SLOT, DEV_BAD_LENGTH, DEV_TIMEOUT, DEV_BAD_PREFIX = 0x1, 0x2, 0x4, 0x8, 0x10
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
     L.pkv_pool_bytes.argtypes = [P, P]
     L.kv_pool_create.restype = i32
     L.kv_pool_create.argtypes = [P, P]
+    L.kv_pool_create_layers.restype = i32
+    L.kv_pool_create_layers.argtypes = [P, P, P, P, P, P]
     L.kv_pool_destroy.restype = i32
     L.kv_pool_destroy.argtypes = [P]
     L.kv_append_workspace_bytes.restype = sz
@@ -99,6 +102,10 @@ def lib() -> ctypes.CDLL:
     L.paged_prefill_chunk_attn_window.argtypes = [P, i32, P, i32, P, i32, i32, i32, i32, f32, i32, P, P]
     L.pkv_read_device_status.restype = i32
     L.pkv_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    L.pkv_get_device_status.restype = i32
+    L.pkv_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+    L.pkv_test_withhold_copy.restype = i32
+    L.pkv_test_withhold_copy.argtypes = [i32, ctypes.c_longlong]
     _lib = L
     return L
 
@@ -161,6 +168,32 @@ class KVPool:
         h = ctypes.c_void_p()
         _check(lib().kv_pool_create(ctypes.byref(self._desc), ctypes.byref(h)), "kv_pool_create")
         self.handle = h
+
+    @classmethod
+    def from_layers(cls, k_layers, v_layers, kv_dtype: int, head_dim: int, k_scales=None, v_scales=None,
+                    device_status=None) -> "KVPool":
+        """A handle over per-layer allocations (kv_pool_create_layers): k_layers[l] / v_layers[l]
+        [N, H_kv, 16, row] tensors, k_scales[l] / v_scales[l] fp32 [N, H_kv] (quantized)."""
+        L = len(k_layers)
+        if L == 0 or len(v_layers) != L or any(t.dim() != 4 or t.shape != k_layers[0].shape
+                                                 for t in list(k_layers) + list(v_layers)):
+            raise ValueError("k_layers / v_layers must be equal-shaped [N, H_kv, 16, row] tensors")
+        self = cls.__new__(cls)
+        N, H, bs, _ = k_layers[0].shape
+        self.k_data, self.v_data = list(k_layers), list(v_layers)
+        self.k_scale = None if k_scales is None else list(k_scales)
+        self.v_scale = None if v_scales is None else list(v_scales)
+        self.device_status = device_status
+        self.num_layers, self.num_blocks, self.num_kv_heads, self.head_dim = L, N, H, head_dim
+        self.kv_dtype = kv_dtype
+        self._desc = _PoolDesc(L, N, bs, H, head_dim, kv_dtype, None, None, None, None, _ptr(device_status))
+        arr = lambda ts: None if ts is None else (ctypes.c_void_p * L)(*[_ptr(t) for t in ts])  # noqa: E731
+        self._arrays = (arr(self.k_data), arr(self.v_data), arr(self.k_scale), arr(self.v_scale))
+        h = ctypes.c_void_p()
+        _check(lib().kv_pool_create_layers(ctypes.byref(self._desc), *self._arrays, ctypes.byref(h)),
+               "kv_pool_create_layers")
+        self.handle = h
+        return self
 
     @classmethod
     def allocate(cls, num_layers: int, num_blocks: int, num_kv_heads: int, head_dim: int, kv_dtype: int,
@@ -366,6 +399,21 @@ def read_device_status(pool: KVPool, stream=None) -> int:
     if rc not in (0, -7, -8):
         _check(rc, "pkv_read_device_status")
     return int(st.value)
+
+
+def get_device_status(pool: KVPool, stream=None) -> tuple[int, int]:
+    """pkv_get_device_status: (its return code, the status bits it read and cleared)."""
+    st = ctypes.c_int32(0)
+    rc = lib().pkv_get_device_status(pool.handle, _stream(stream), ctypes.byref(st))
+    if rc not in (0, -7, -8):
+        _check(rc, "pkv_get_device_status")
+    return int(rc), int(st.value)
+
+
+def test_withhold_copy(tile: int, wait_cycles: int = 0) -> None:
+    """pkv_test_withhold_copy: from now on every attention kernel withholds the copy of its
+    `tile`-th K/V tile and bounds its waits at `wait_cycles` SM cycles (tile < 0: off)."""
+    _check(lib().pkv_test_withhold_copy(int(tile), int(wait_cycles)), "pkv_test_withhold_copy")
 
 
 # ------------------------------------------------------------ block manager --

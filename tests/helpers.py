@@ -4,6 +4,9 @@ Nothing here computes attention or quantization; it only copies the same input b
 both sides and, for full-size workloads, gives the oracle a compact copy of just the
 blocks a sampled subset of sequences references (block ids renumbered).
 """
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -42,3 +45,42 @@ def max_abs_diff(gpu_out: torch.Tensor, ref: np.ndarray) -> float:
     assert g.shape == ref.shape, (g.shape, ref.shape)
     assert np.isfinite(g).all(), "non-finite GPU output"
     return float(np.abs(g - ref).max()) if g.size else 0.0
+
+
+def host_threads(cap: int = 64) -> int:
+    """Host cores this process may run on (at most `cap`)."""
+    n = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    return max(1, min(n, cap))
+
+
+def oracle_decode_threaded(opool, q, q_dtype, tables, ctx_lens, scale, window: int = 0) -> np.ndarray:
+    """oracle.paged_decode with the sequences split over host threads.  Each sequence is
+    computed on its own in the oracle, so the result is the one a single call gives; the
+    C oracle runs without the GIL (ctypes releases it)."""
+    B = q.shape[0]
+    tables = torch.as_tensor(tables)
+    ctx_lens = torch.as_tensor(ctx_lens)
+    n = min(host_threads(), max(1, B))
+    bounds = [B * i // n for i in range(n + 1)]
+
+    def part(i):
+        a, b = bounds[i], bounds[i + 1]
+        if a == b:
+            return np.zeros((0,) + tuple(q.shape[1:]), np.float64)
+        return oracle.paged_decode(opool, q[a:b], q_dtype, tables[a:b], ctx_lens[a:b], scale, window=window)
+
+    with ThreadPoolExecutor(n) as ex:
+        return np.concatenate(list(ex.map(part, range(n))))
+
+
+def oracle_chunk_threaded(opool, q, q_dtype, block_table, ctx_before: int, scale, rows) -> np.ndarray:
+    """oracle.paged_prefill_chunk for the listed chunk rows, over host threads.  Row i of a
+    chunk after ctx_before positions is row 0 of a one-row chunk after ctx_before + i
+    positions (the same keys, the same causal bound), so each row is its own oracle call."""
+    rows = list(rows)
+
+    def one(i):
+        return oracle.paged_prefill_chunk(opool, q[i:i + 1], q_dtype, block_table, ctx_before + i, scale)[0]
+
+    with ThreadPoolExecutor(host_threads()) as ex:
+        return np.stack(list(ex.map(one, rows)))

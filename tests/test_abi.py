@@ -176,6 +176,14 @@ def _decode_ws(h, B, H_q, ctx, opts=None):
     return pkv.lib().paged_decode_workspace_bytes(h, B, H_q, ctx, ctypes.byref(opts) if opts is not None else None)
 
 
+def _ws_expected(B, H_q, H_kv, parts, d=128):
+    """fp32 partials o[d] + (m, l) per (sequence, query head, partition), then one int32 merge
+    counter per (sequence, KV head, group of 16 query heads); nothing for one partition."""
+    if parts <= 1:
+        return 0
+    return B * H_q * parts * (d + 2) * 4 + B * H_kv * (-(-(H_q // H_kv) // 16)) * 4
+
+
 @pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 1024), (pkv.FP8E4M3, 1024),
                                      (pkv.INT4, 2048)])
 def test_decode_workspace_follows_the_partition_policy(dtype, P):
@@ -189,10 +197,10 @@ def test_decode_workspace_follows_the_partition_policy(dtype, P):
     assert rc == 0
     try:
         B, H_q, ctx = 170, 64, 8192
-        assert _decode_ws(h, B, H_q, ctx) == B * H_q * (-(-ctx // P)) * (128 + 2) * 4
+        assert _decode_ws(h, B, H_q, ctx) == _ws_expected(B, H_q, 8, -(-ctx // P))
         # a context of one default partition: with only B * H_kv CTAs the grid cannot fill the GPU, so
         # partitions are halved (to 128 tokens at least) and the partials come back
-        short = _decode_ws(h, B, H_q, P)
+        short = _decode_ws(h, B, H_q, P) - _ws_expected(B, H_q, 8, 2) + B * H_q * 2 * (128 + 2) * 4
         parts, rem = divmod(short, B * H_q * (128 + 2) * 4)
         assert rem == 0 and 2 <= parts <= P // 128 and parts & (parts - 1) == 0
         assert _decode_ws(h, B, H_q, 128) == 0                         # one partition: no partials
@@ -204,15 +212,68 @@ def test_decode_workspace_small_batches_and_explicit_partitions():
     rc, h = _create(num_kv_heads=8, head_dim=128, kv_dtype=pkv.BF16)
     assert rc == 0
     try:
-        row = (128 + 2) * 4
         # 2 sequences cannot fill 148 SMs with 512-token partitions: they shrink to the 128-token floor
-        assert _decode_ws(h, 2, 64, 8192) == 2 * 64 * 64 * row
+        assert _decode_ws(h, 2, 64, 8192) == _ws_expected(2, 64, 8, 64)
         # an explicit partition size is taken as given (a multiple of 16 in [64, 4096])
-        assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, 64, 0)) == 3 * 16 * 16 * row
+        assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, 64, 0)) == _ws_expected(3, 16, 8, 16)
         assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, 4096, 0)) == 0
         for bad in (100, 48, 8192):
             assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, bad, 0)) == 0
-        # the partials scale with the batch and the query heads, not with the KV heads' grouping
+        # the workspace scales with the batch
         assert _decode_ws(h, 340, 64, 8192) == 2 * _decode_ws(h, 170, 64, 8192)
+        # wide groups: one counter per 16 query heads of a KV head
+        assert _decode_ws(h, 3, 8 * 40, 1000, pkv._DecodeOpts(0, 64, 0)) == _ws_expected(3, 320, 8, 16)
     finally:
         pkv.lib().kv_pool_destroy(h)
+
+
+def test_wait_hook_arguments_are_checked_on_the_host():
+    """pkv_test_withhold_copy only stores process-wide settings; out-of-range bounds are
+    rejected and tile < 0 restores the defaults (no CUDA call)."""
+    L = pkv.lib()
+    assert L.pkv_test_withhold_copy(0, 0) == -2
+    assert L.pkv_test_withhold_copy(0, 3_000_000_000) == -2
+    assert L.pkv_test_withhold_copy(1, 100_000) == 0
+    assert L.pkv_test_withhold_copy(-1, 0) == 0
+
+
+def test_get_device_status_is_read_device_status():
+    """Both names validate the same way before touching the device."""
+    L = pkv.lib()
+    st = ctypes.c_int32(5)
+    assert L.pkv_get_device_status(None, None, ctypes.byref(st)) == -1
+    assert L.pkv_read_device_status(None, None, ctypes.byref(st)) == -1
+
+
+def test_per_layer_pool_create_validation():
+    """kv_pool_create_layers checks every layer's pointers on the host (no CUDA call): NULL
+    arrays or entries, misaligned bases, missing scales of a quantized pool, too many layers."""
+    L = pkv.lib()
+    P = ctypes.c_void_p
+
+    def arr(vals):
+        return (P * len(vals))(*vals)
+
+    def create(desc, k, v, ks=None, vs=None):
+        h = ctypes.c_void_p()
+        rc = L.kv_pool_create_layers(ctypes.byref(desc), k, v, ks, vs, ctypes.byref(h))
+        if rc == 0:
+            assert h.value and L.kv_pool_destroy(h) == 0
+        return rc
+
+    d3 = _desc(num_layers=3, k_data=None, v_data=None)
+    k = arr([0x100000, 0x900000, 0x500000])          # any order, any spacing
+    v = arr([0x200000, 0x300000, 0x700000])
+    assert create(d3, k, v) == 0
+    assert create(d3, None, v) == -1
+    assert create(d3, k, arr([0x200000, None, 0x700000])) == -1
+    assert create(d3, k, arr([0x200000, 0x300008, 0x700000])) == -2      # not 16-byte aligned
+    q3 = _desc(num_layers=3, kv_dtype=pkv.INT8, k_data=None, v_data=None)
+    assert create(q3, k, v) == -1                                        # quantized without scales
+    s = arr([0x1000, 0x2000, 0x3000])
+    assert create(q3, k, v, s, arr([0x4000, 0x5000, 0x6000])) == 0
+    assert create(q3, k, v, s, arr([0x4000, 0x5002, 0x6000])) == -2     # scales not 4-byte aligned
+    big = _desc(num_layers=pkv.MAX_LAYERS + 1, k_data=None, v_data=None)
+    many = arr([0x100000] * (pkv.MAX_LAYERS + 1))
+    assert create(big, many, many) == -2
+    assert _create(num_layers=pkv.MAX_LAYERS + 1)[0] == -2

@@ -37,3 +37,18 @@ def test_reference_arm_line(workload, threads):
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_wave_reports_a_failed_thread(monkeypatch):
+    """A host thread whose oracle call raises ends the wave with that thread's own error
+    (the other threads are released from the barriers and joined)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+
+    def failing(*args, **kw):
+        raise ValueError("planted failure in one oracle call")
+
+    monkeypatch.setattr(oracle, "paged_decode", failing)
+    with pytest.raises(RuntimeError, match="planted failure"):
+        bench.cpu_oracle_waves("mqa", steps=1, warmup=0, max_threads=2)

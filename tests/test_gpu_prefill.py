@@ -7,7 +7,7 @@ import torch
 import oracle
 from paged_kv_cache_431_b200 import pkv
 from paged_kv_cache_431_b200 import workloads as wl
-from tests.helpers import TOL, compact_subset, max_abs_diff, oracle_pool_from_tensors, oracle_subset_pool
+from tests.helpers import TOL, max_abs_diff, oracle_chunk_threaded, oracle_pool_from_tensors
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -66,7 +66,7 @@ def test_chunk_parity(case):
 
 def test_prefix_plus_chunk_config():
     """One layer of the 70B shape: a 4,000-token shared prefix (250 blocks) and a 512-token
-    chunk appended after it, then the chunk attends to prefix + itself."""
+    chunk appended after it, then the chunk attends to prefix + itself; every row checked."""
     g = wl.generator(435)
     H_q, H_kv, d, P0, C = 64, 8, 128, 4000, 512
     N = 250 + 32 + 64
@@ -86,11 +86,9 @@ def test_prefix_plus_chunk_config():
     torch.cuda.synchronize()
     assert pkv.read_device_status(pool) == 0
     oracle.kv_append(opool, k_new.cpu(), v_new.cpu(), wl.BF16, slots.numpy())
-    rows = [0, 1, 255, 511]
-    ref = oracle.paged_prefill_chunk(opool, q[rows[0]:rows[0] + 1].cpu(), wl.BF16, paging.tables[0], P0,
-                                     np.float32(d ** -0.5))
-    assert max_abs_diff(out[0:1], ref) <= TOL
-    for i in rows[1:]:
-        ref = oracle.paged_decode(opool, q[i:i + 1].cpu(), wl.BF16, paging.tables[0:1],
-                                  [P0 + i + 1], np.float32(d ** -0.5))
-        assert max_abs_diff(out[i:i + 1], ref) <= TOL
+    # every row of the chunk (all 32 query tiles of the kernel), the oracle on all host cores
+    ref = oracle_chunk_threaded(opool, q.cpu(), wl.BF16, paging.tables[0], P0, np.float32(d ** -0.5), range(C))
+    assert max_abs_diff(out, ref) <= TOL
+    # and the first rows through the oracle's own multi-row chunk form
+    ref = oracle.paged_prefill_chunk(opool, q[:3].cpu(), wl.BF16, paging.tables[0], P0, np.float32(d ** -0.5))
+    assert max_abs_diff(out[:3], ref) <= TOL

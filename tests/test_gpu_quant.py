@@ -8,7 +8,7 @@ import torch
 import oracle
 from paged_kv_cache_431_b200 import pkv
 from paged_kv_cache_431_b200 import workloads as wl
-from tests.helpers import TOL, max_abs_diff
+from tests.helpers import TOL, max_abs_diff, oracle_decode_threaded
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -156,7 +156,8 @@ def test_quantized_decode_parity(dt, case):
 def test_quantized_long_context_config(dt):
     """Quantized long-context decode, 1 layer: B 16, H_q 64, H_kv 8, d 128, contexts
     U[32768, 131072], bf16 N(0, 1) source with 1% outlier channels x8, bulk-filled by
-    kv_append; the oracle checks the codes and the outputs of 2 sampled sequences."""
+    kv_append; the oracle checks the codes and the outputs of 4 sampled sequences (the
+    shortest and 3 seeded others)."""
     g = wl.generator(436)
     B, H_q, H_kv, d = 16, 64, 8, 128
     ctx = wl.quant_long_lens(g, B)
@@ -165,9 +166,8 @@ def test_quantized_long_context_config(dt):
     paging = wl.allocate(ctx, N, W, g)
     out_ch = wl.outlier_channels(g, H_kv, d)
     pool = pkv.KVPool.allocate(1, N, H_kv, d, dt)
-    sampled = [int(torch.argmin(ctx)), int(torch.randint(0, B, (1,), generator=g))]
-    if sampled[1] == sampled[0]:
-        sampled[1] = (sampled[0] + 1) % B
+    shortest = int(torch.argmin(ctx))
+    sampled = [shortest] + [b for b in torch.randperm(B, generator=g).tolist() if b != shortest][:3]
     gd = wl.generator(437, DEV)
     host_src = {}
     for b in range(B):
@@ -192,12 +192,12 @@ def test_quantized_long_context_config(dt):
     assert np.array_equal(pool.k_data[0][idx].cpu().numpy().reshape(opool.k.shape), opool.k)
     assert np.array_equal(pool.v_data[0][idx].cpu().numpy().reshape(opool.v.shape), opool.v)
     assert np.array_equal(pool.k_scale[0][idx].cpu().numpy(), opool.k_scale)
-    ref = oracle.paged_decode(opool, q[sampled].cpu(), oracle.BF16, sub_t, sub_c, np.float32(d ** -0.5))
+    ref = oracle_decode_threaded(opool, q[sampled].cpu(), oracle.BF16, sub_t, sub_c, np.float32(d ** -0.5))
     assert max_abs_diff(out[sampled], ref) <= TOL
 
 
-# q magnitudes: the integer-code kernels pre-scale q by a power of two chosen per CTA
-# from its largest |q| (and treat all-zero q separately); the fp8 kernel does not.
+# q magnitudes: every quantized kernel pre-scales q by a power of two chosen per CTA from its
+# largest |q| before converting it to fp16 (all-zero q takes the largest shift).
 Q_MAGNITUDES = {
     "zero": lambda q: q * 0,                 # every score 0: out = mean of the dequantized V
     "tiny": lambda q: q * 1e-3,              # q near the bottom of fp16's normal range
@@ -236,3 +236,68 @@ def test_quantized_decode_query_magnitudes(dt, mag):
             rows = vdq[paging.tables[b].numpy()[t // 16], :, t % 16, :]      # [n, H_kv, d]
             want = np.repeat(rows.mean(axis=0), G, axis=0)                     # [H_q, d]
             assert np.abs(out[b].cpu().double().numpy() - want).max() <= TOL
+
+
+# q shapes that stress the score arithmetic of the quantized kernels at long contexts:
+#   same_sign -- every q_d > 0: the integer-code kernels add offset * sum(q) to the raw
+#                scores and take it off again; with one sign that share is ~20x the score;
+#   constant  -- q_d = 0.75 for every d and head: the same offset share, and every head
+#                of a group computes the same scores;
+#   huge      -- max |q| = 1e5 (bf16 holds it, fp16 does not): q of head h is the bf16 K
+#                source of one token t_b of the sequence, scaled up; without outlier channels
+#                q . k_t is ~128 x the scale and any other key's ~N(0, 128) x the scale, so the
+#                softmax is one-hot at t_b by thousands of log2 units (no near-tie for
+#                rounding to flip) and the output is that token's dequantized V row;
+#   small     -- |q| ~ 1e-6 (below fp16's normal range): near-uniform weights.
+Q_STRESS = ("same_sign", "constant", "huge", "small")
+
+
+def stress_q(mag, q, k_src, lens, G):
+    """q [B, H_q, d] fp32 N(0, 1) -> the stressing form; k_src [sum(lens), H_kv, d] bf16."""
+    if mag == "same_sign":
+        return q.abs()
+    if mag == "constant":
+        return torch.full_like(q, 0.75)
+    if mag == "small":
+        return q * 1e-6
+    starts = np.cumsum([0] + list(lens[:-1]))
+    for b, n in enumerate(lens):
+        t = (n * 2) // 3                                   # the token each head aligns with
+        q[b] = k_src[starts[b] + t].float().repeat_interleave(G, dim=0)
+    return q * (1e5 / q.abs().max())
+
+
+@pytest.mark.parametrize("mag", Q_STRESS)
+@pytest.mark.parametrize("dt", QDTYPES, ids=lambda x: NAMES[x])
+def test_quantized_decode_query_stress_long_context(dt, mag):
+    """The 70B head shape (H_q 64, H_kv 8, d 128) at contexts of 1,000-4,100 tokens (split-K
+    partitions of 1,024 / 2,048 tokens, plus one short sequence), with the stressing q
+    shapes above, against the oracle at 2e-3."""
+    H_q, H_kv, d = 64, 8, 128
+    g = wl.generator(1300 + 10 * dt + Q_STRESS.index(mag))
+    lens = [1000, 1777, 3000, 4100, 33]
+    N = sum(wl.ceil_div(n, 16) for n in lens) + 3
+    paging = wl.allocate(lens, N, 260, g)
+    pool = pkv.KVPool.allocate(1, N, H_kv, d, dt)
+    seq = torch.cat([torch.full((n,), b) for b, n in enumerate(lens)])
+    pos = torch.cat([torch.arange(n) for n in lens])
+    slots = wl.slots_for(paging.tables, seq, pos)
+    out_ch = wl.outlier_channels(g, H_kv, d)
+    k, v = wl.kv_source(len(seq), H_kv, d, g, outliers=None if mag == "huge" else out_ch)
+    pkv.kv_append(pool, 0, k.to(DEV), v.to(DEV), slots.to(DEV))
+    opool = oracle_copy(pool)
+    q = stress_q(mag, wl.normal((len(lens), H_q, d), torch.float32, g), k, lens, H_q // H_kv).to(torch.bfloat16)
+    if mag == "huge":
+        assert q.float().abs().max().item() > 65504.0      # outside fp16's range
+    out = pkv.paged_decode_attn(pool, 0, q.to(DEV), paging.tables.to(DEV), paging.ctx_lens.to(DEV), d ** -0.5,
+                                max(lens))
+    torch.cuda.synchronize()
+    assert pkv.read_device_status(pool) == 0
+    ref = oracle_decode_threaded(opool, q, oracle.BF16, paging.tables, paging.ctx_lens, np.float32(d ** -0.5))
+    assert max_abs_diff(out, ref) <= TOL
+    if mag == "huge":   # one-hot: the aligned token's dequantized V row (oracle side, fp64)
+        vdq = opool.dequant("v")
+        for b, n in enumerate(lens):
+            t = (n * 2) // 3
+            row = np.repeat(vdq[int(paging.tables[b, t // 16]), :, t % 16, :], H_q // H_kv, axis=0)
+            assert np.abs(ref[b] - row).max() <= 1e-9

@@ -15,26 +15,43 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def decode_inputs(seed, B, H_q, H_kv, d):
+def decode_inputs(seed, B, H_q, H_kv, d, kv_dtype=wl.BF16):
     g = wl.generator(seed)
     ctx = wl.llama8b_lens(g, B)
     N = B * 4096 // 16
     paging = wl.allocate(ctx, N, 256, g)
     gd = wl.generator(seed + 1, DEV)
-    k = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, DEV)
-    v = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, DEV)
+    if kv_dtype == wl.BF16:
+        k = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, DEV)
+        v = wl.normal((1, N, H_kv, 16, d), torch.bfloat16, gd, DEV)
+        pool = pkv.KVPool(k, v, wl.BF16, d, device_status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    else:   # a quantized pool filled through kv_append
+        pool = pkv.KVPool.allocate(1, N, H_kv, d, kv_dtype)
+        for b in range(B):
+            n = int(ctx[b])
+            k, v = wl.kv_source(n, H_kv, d, gd, DEV)
+            pkv.kv_append(pool, 0, k, v, wl.slots_for(paging.tables, [b] * n, torch.arange(n)).to(DEV))
     q = wl.normal((B, H_q, d), torch.bfloat16, gd, DEV)
-    pool = pkv.KVPool(k, v, wl.BF16, d, device_status=torch.zeros(1, dtype=torch.int32, device=DEV))
     return pool, q, paging.tables.to(DEV), ctx.to(DEV), int(ctx.max())
 
 
-def test_noalloc_matches_regular_decode_on_two_calls():
+CASES = {
+    # name: (pool dtype, sliding window)
+    "bf16": (wl.BF16, 0),
+    "int8": (wl.INT8, 0),
+    "bf16_window": (wl.BF16, 1000),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_noalloc_matches_regular_decode_on_two_calls(name):
+    kv_dtype, window = CASES[name]
     for seed, B in ((801, 64), (802, 24)):
-        pool, q, tables, ctx, max_ctx = decode_inputs(seed, B, 32, 8, 128)
-        need = pkv.paged_decode_workspace_bytes(pool, B, 32, max_ctx)
+        pool, q, tables, ctx, max_ctx = decode_inputs(seed, B, 32, 8, 128, kv_dtype)
+        need = pkv.paged_decode_workspace_bytes(pool, B, 32, max_ctx, sliding_window=window)
         assert 0 < need <= pkv.NOALLOC_SCRATCH_BYTES          # the split-K path is exercised
-        ref = pkv.paged_decode_attn(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx)
-        out = pkv.paged_decode_attn_noalloc(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx)
+        ref = pkv.paged_decode_attn(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx, sliding_window=window)
+        out = pkv.paged_decode_attn_noalloc(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx, sliding_window=window)
         torch.cuda.synchronize()
         assert pkv.read_device_status(pool) == 0
         assert torch.isfinite(out).all()
