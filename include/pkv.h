@@ -179,10 +179,9 @@ typedef struct {
 } pkv_decode_opts;
 
 /* Workspace paged_decode_attn needs for these sizes and options (bytes): per (sequence,
- * query head, partition) a head_dim + 2 fp32 partial (o, m, l), then one int32 merge counter
- * per (sequence, KV head, group of 16 query heads), which every call clears itself (one
- * cudaMemsetAsync); 0 when every sequence fits one partition.
- * With a sliding window the partitions cover at most window + 15 tokens per sequence. */
+ * query head, partition) a head_dim + 2 fp32 partial (o, m, l); 0 when every sequence fits
+ * one partition.  With a sliding window the partitions cover at most window + 15 tokens per
+ * sequence. */
 PKV_API size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads,
                                     int max_context_len, const pkv_decode_opts* opts);
 
@@ -229,8 +228,8 @@ PKV_API int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_d
  * The first call on a device looks up the buffer's device address (cudaGetSymbolAddress,
  * with that device current); make that first call before any stream capture on the device.
  * All calls share the buffer and it keeps the last call's contents (no call relies on them:
- * each writes every partial it reads and clears the merge counters it uses).  Calls whose
- * kernels may overlap on the GPU race on the buffer; issue them in order on one stream.
+ * each writes every partial it reads).  Calls whose kernels may overlap on the GPU race on
+ * the buffer; issue them in order on one stream.
  */
 PKV_API int paged_decode_attn_noalloc(pkv_pool_t pool, int layer, const void* q, int q_dtype,
                                       const int32_t* block_tables, int block_table_width,

@@ -328,13 +328,11 @@ static int decode_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, i
     return PKV_OK;
 }
 
-// Split-K workspace: partials o [B][H_q][parts][d] and (m, l) [B][H_q][parts][2] (fp32), then
-// one int counter per (sequence, CTA of a partition) for the fused merge.
+// Split-K workspace: partials o [B][H_q][parts][d] and (m, l) [B][H_q][parts][2] (fp32).
 static size_t decode_ws_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int parts)
 {
     if (parts <= 1) return 0;
-    return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float) +
-           (size_t)num_seqs * ctas_per_partition(pool, num_q_heads) * sizeof(int);
+    return (size_t)num_seqs * num_q_heads * parts * (pool->d.head_dim + 2) * sizeof(float);
 }
 
 size_t paged_decode_workspace_bytes(pkv_pool_t pool, int num_seqs, int num_q_heads, int max_context_len,
@@ -399,9 +397,6 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     float* ws = static_cast<float*>(workspace);
     a.ws_o = need ? ws : nullptr;
     a.ws_ml = need ? ws + (size_t)num_seqs * num_q_heads * parts * d.head_dim : nullptr;
-    a.counters = need ? reinterpret_cast<int*>(ws + (size_t)num_seqs * num_q_heads * parts * (d.head_dim + 2))
-                      : nullptr;
-    a.counter_count = need ? num_seqs * ctas_per_partition(pool, num_q_heads) : 0;
     a.status = d.device_status;
     a.engine = engine;
     a.window = opts ? opts->sliding_window : 0;

@@ -28,11 +28,9 @@
 //     shuffles.  Masked (past-the-end) tokens get -inf scores and zeroed V, so stale or
 //     poisoned slots never reach the result.
 //   * Split-K: a sequence longer than one partition writes per-partition (o, m, l)
-//     partials and counts itself done on a per-(sequence, head group) counter; the CTA that
-//     completes the count merges them with the log-sum-exp rule (no second launch).  The
-//     shared-prefix (cascade) form starts the partitions after the prefix and leaves the
-//     merge, with the prefix's partials written by the tensor-core prefill kernel, to
-//     decode_reduce.
+//     partials; decode_reduce merges them with the log-sum-exp rule.  The shared-prefix
+//     (cascade) form starts the partitions after the prefix and merges them with the
+//     prefix's partials written by the tensor-core prefill kernel.
 #include "decode_common.cuh"
 
 namespace pkv {
@@ -349,10 +347,6 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 }
             }
         }
-        if (p.counters) {   // the CTA that completes this (sequence, head group) merges all partitions
-            __shared__ int s_last;
-            if (last_partition(p, b, nparts, &s_last)) merge_partials<D>(p, row0, GC, nparts, lane);
-        }
     }
 }
 
@@ -466,7 +460,6 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.out = a.out;
     p.ws_o = a.ws_o;
     p.ws_ml = a.ws_ml;
-    p.counters = nullptr;
     p.status = a.status;
     p.W = a.W;
     p.H_q = a.H_q;
@@ -489,15 +482,6 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
 
     const dim3 grid(a.max_parts, a.H_kv * p.hgroups, a.B);
     const int nht = a.G <= 8 ? 1 : 2;   // 8 or 16 query heads per CTA
-    // The tensor-core engines merge the split-K partials in the CTA that finishes a
-    // (sequence, head group) last; its counters start at zero (one small memset per call: the
-    // workspace is the caller's and may hold anything).  The CUDA-core engines and the cascade
-    // form merge in decode_reduce.
-    if (a.counters && a.max_parts > 1 && a.part_base == 0 && a.engine == 1) {
-        if (cudaMemsetAsync(a.counters, 0, (size_t)a.counter_count * sizeof(int), s) != cudaSuccess)
-            return PKV_ERR_CUDA;
-        p.counters = a.counters;
-    }
     int rc = PKV_ERR_UNSUPPORTED;
     if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && (a.engine == 2 || a.engine == 3)) {
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
@@ -515,7 +499,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         rc = launch_decode_quant(p, a.kv_dtype, a.d, nht, grid, s, tmk, tmv);
     }
     if (rc != PKV_OK) return rc;
-    if ((a.max_parts > 1 && !p.counters) || a.part_base > 0) {
+    if (a.max_parts > 1 || a.part_base > 0) {
         // programmatic dependent launch: scheduled while the decode grid's last wave runs
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(a.H_q, a.B);

@@ -18,8 +18,6 @@ struct DecodeParams {
     float* out;
     float* ws_o;
     float* ws_ml;
-    int* counters;          // fused merge: one per (sequence, CTA row of the grid), zero at entry; null:
-                            // the separate decode_reduce_kernel merges (cascade, CUDA-core engines)
     int32_t* status;
     int W, H_q, H_kv, G, N, part_tokens, max_parts;
     // Partitions cover tokens tok_base .. ctx-1 and write workspace slots part_base + part of
@@ -71,74 +69,6 @@ __device__ __forceinline__ int part_count(const DecodeParams& p, int ctx)
 __device__ __forceinline__ size_t ws_slot(const DecodeParams& p, size_t row, int part)
 {
     return row * p.slots + p.part_base + part;
-}
-
-// Split-K merge of the partials of query heads row0 .. row0 + nh - 1 (rows b * H_q + h) over
-// partitions 0 .. nparts-1 of this launch, by one warp:
-//   out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,  M = max_i m_i  (log2-domain m).
-// The partials were written by other CTAs: loads bypass L1 (ld.global.cg).
-template <int D>
-__device__ __forceinline__ void merge_partials(const DecodeParams& p, size_t row0, int nh, int nparts, int lane)
-{
-    constexpr int V = D / 32;   // floats per lane
-    for (int h = 0; h < nh; ++h) {
-        const size_t base = (row0 + h) * p.slots + p.part_base;
-        const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + base;
-        float M = -INFINITY;
-        for (int i = lane; i < nparts; i += 32) M = fmaxf(M, __ldcg(&ml[i]).x);
-#pragma unroll
-        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float L = 0.f;
-        for (int i = lane; i < nparts; i += 32) {
-            const float2 v = __ldcg(&ml[i]);
-            L += ex2(v.x - M) * v.y;
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        float acc[V];
-#pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = 0.f;
-        const float* po = p.ws_o + base * D + lane * V;
-#pragma unroll 4
-        for (int i = 0; i < nparts; ++i) {
-            const float w = ex2(__ldcg(&ml[i]).x - M);
-            if constexpr (V == 4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(po + (size_t)i * D));
-                acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-            } else {
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(po + (size_t)i * D));
-                acc[0] += w * v.x; acc[1] += w * v.y;
-            }
-        }
-        const float inv = 1.f / L;
-        float* o = p.out + (row0 + h) * D + lane * V;
-        if constexpr (V == 4) {
-            *reinterpret_cast<float4*>(o) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-        } else {
-            *reinterpret_cast<float2*>(o) = make_float2(acc[0] * inv, acc[1] * inv);
-        }
-    }
-}
-
-// After this CTA's partials are written: count the partition done; true in the CTA that
-// completes the (sequence, CTA row) -- it then merges, and leaves the counter at zero for the
-// next call.  Every thread of the CTA calls it (one warp: `lane`-uniform; several warps: a CTA
-// barrier inside); all return the same value.
-__device__ __forceinline__ bool last_partition(const DecodeParams& p, int b, int nparts, int* s_flag)
-{
-    __threadfence();   // this thread's partial stores are visible device-wide before the count
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int* c = p.counters + (size_t)b * gridDim.y + blockIdx.y;
-        const int done = atomicAdd(c, 1) + 1;
-        const bool last = done == nparts;
-        if (last) atomicExch(c, 0);
-        *s_flag = last;
-    }
-    __syncthreads();
-    const bool last = *s_flag;
-    if (last) __threadfence();   // the other CTAs' partials are read after their counts
-    return last;
 }
 
 // Byte address of 16-byte chunk `c` of row `t` in a tile stored as 128-byte-wide TMA

@@ -573,10 +573,6 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
                     make_float2(m_run[hr], l_run[hr]);
         }
     }
-    if (!final_out && p.counters) {   // the CTA that completes this (sequence, head group) merges
-        __shared__ int s_last;
-        if (last_partition(p, b, nparts, &s_last)) merge_partials<D>(p, row0, GC, nparts, lane);
-    }
 }
 
 template <int DT, int D>

@@ -59,8 +59,6 @@ struct DecodeArgs {
     float* out;
     float* ws_o;            // [B][H_q][max_parts][d]
     float* ws_ml;           // [B][H_q][max_parts][2]
-    int* counters = nullptr;    // fused split-K merge: counter_count ints after the partials
-    int counter_count = 0;
     int32_t* status;
     int engine;             // 1 mma, 2 fma
     int tok_base = 0;       // first token the partitions cover (cascade: the prefix length)

@@ -16,11 +16,10 @@
 // device current -- and that address is passed to the kernels.
 //
 // All calls on a device share the one buffer and it keeps the last call's contents.
-// A call writes every partial it later reads; the one part that must start at zero, the
-// split-K merge counters, is cleared by every call itself (a cudaMemsetAsync, which
-// allocates nothing).  Two calls whose kernels overlap on the GPU (different streams, or
-// different host threads, without ordering between them) race on the buffer and give wrong
-// results; callers must serialize them, e.g. by issuing them on one stream.
+// Nothing in it has to start at zero: a call writes every partial it later reads.  Two
+// calls whose kernels overlap on the GPU (different streams, or different host threads,
+// without ordering between them) race on the buffer and give wrong results; callers must
+// serialize them, e.g. by issuing them on one stream.
 #include <mutex>
 
 #include "internal.h"

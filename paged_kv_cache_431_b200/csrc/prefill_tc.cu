@@ -161,6 +161,13 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -182,6 +189,14 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
     *abort_flag = 1;
     flag_status(status, PKV_DEV_TIMEOUT);
     return false;
+}
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 // Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction.
@@ -450,23 +465,29 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 break;
             }
             tc_fence_after();
-            // pass 1: the row maximum over the tile's 128 scores (64 at a time)
+            // the row's 128 scores of this key tile, read from TMEM once
             const int key0 = (t_lo + t) * kBN;
             const bool need_mask = key0 + kBN > kmin_tile;
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
+            float v[kBN];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[64];
-                tmem_ld32(tS + 64 * hh, *reinterpret_cast<float(*)[32]>(&v[0]));
-                tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-                tmem_wait_ld();
+            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(&v[32 * c]));
+            tmem_wait_ld();
+            if (!pos_scale) {   // a scale <= 0: apply it before the maximum (slx is then 1)
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float xj = (need_mask && key0 + 64 * hh + j >= kmax) ? -INFINITY : v[j];
-                    m4[j & 3] = fmaxf(m4[j & 3], pos_scale ? xj : xj * sl);
-                }
+                for (int j = 0; j < kBN; ++j) v[j] *= sl;
             }
-            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if (need_mask) {
+#pragma unroll
+                for (int j = 0; j < kBN; ++j)
+                    if (key0 + j >= kmax) v[j] = -INFINITY;
+            }
+            // row maximum: three-input maxima in four independent chains
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int j = 0; j < kBN; j += 8)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[j + 2 * k], v[j + 2 * k + 1]);
+            float mx = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], -INFINITY);
             if (pos_scale) mx *= sl;
             float m_new = m_used;
             if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
@@ -475,39 +496,35 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             // keys 32c .. 32c+31 -> columns 32c .. 32c+15 (high), 32c+16 .. 32c+31 (low).
             // bf16: the high part is the truncation (upper half of the fp32 word), the low part
             // the truncated remainder, both by byte permutes.
-            // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             const float2 slx2 = make_float2(slx, slx), mref2 = make_float2(-mref, -mref);
             float2 sum2 = make_float2(0.f, 0.f);
-#pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
-                float v[32];
-                tmem_ld32(tS + 32 * c, v);
-                tmem_wait_ld();
-                if (need_mask) {
+            // 16 keys at a time: keys 32c + 16h .. +15 -> high parts in columns 32c + 8h .. +7,
+            // low parts in columns 32c + 16 + 8h .. +7
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (key0 + 32 * c + j >= kmax) v[j] = -INFINITY;
-                }
-                uint32_t w[32];
+            for (int c16 = 0; c16 < kBN / 16; ++c16) {
+                uint32_t wh[8], wl[8];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 a = ffma2(make_float2(v[2 * e], v[2 * e + 1]), slx2, mref2);
+                for (int e = 0; e < 8; ++e) {
+                    const int j = 16 * c16 + 2 * e;
+                    const float2 a = ffma2(make_float2(v[j], v[j + 1]), slx2, mref2);
                     const float2 pp = make_float2(ex2(a.x), ex2(a.y));
                     if constexpr (BF16) {
                         const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
-                        w[e] = __byte_perm(u0, u1, 0x7632);
+                        wh[e] = __byte_perm(u0, u1, 0x7632);
                         const float2 rr = fsub2(pp, make_float2(__uint_as_float(u0 & 0xffff0000u),
                                                                 __uint_as_float(u1 & 0xffff0000u)));
-                        w[16 + e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+                        wl[e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                     } else {
-                        w[e] = pack2<false>(pp.x, pp.y);
-                        const float2 back = unpack2<false>(w[e]);
-                        w[16 + e] = pack2<false>(pp.x - back.x, pp.y - back.y);
+                        wh[e] = pack2<false>(pp.x, pp.y);
+                        const float2 back = unpack2<false>(wh[e]);
+                        wl[e] = pack2<false>(pp.x - back.x, pp.y - back.y);
                     }
                     sum2 = fadd2(sum2, pp);
                 }
-                tmem_st32u(tS + 32 * c, w);
+                const uint32_t col = 32 * (c16 >> 1) + 8 * (c16 & 1);
+                tmem_st8u(tS + col, wh);
+                tmem_st8u(tS + col + 16, wl);
             }
             l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;

@@ -177,11 +177,11 @@ def _decode_ws(h, B, H_q, ctx, opts=None):
 
 
 def _ws_expected(B, H_q, H_kv, parts, d=128):
-    """fp32 partials o[d] + (m, l) per (sequence, query head, partition), then one int32 merge
-    counter per (sequence, KV head, group of 16 query heads); nothing for one partition."""
+    """fp32 partials o[d] + (m, l) per (sequence, query head, partition); nothing for one
+    partition (H_kv does not enter: the partials are per query head)."""
     if parts <= 1:
         return 0
-    return B * H_q * parts * (d + 2) * 4 + B * H_kv * (-(-(H_q // H_kv) // 16)) * 4
+    return B * H_q * parts * (d + 2) * 4
 
 
 @pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 1024), (pkv.FP8E4M3, 1024),
@@ -221,7 +221,7 @@ def test_decode_workspace_small_batches_and_explicit_partitions():
             assert _decode_ws(h, 3, 16, 1000, pkv._DecodeOpts(0, bad, 0)) == 0
         # the workspace scales with the batch
         assert _decode_ws(h, 340, 64, 8192) == 2 * _decode_ws(h, 170, 64, 8192)
-        # wide groups: one counter per 16 query heads of a KV head
+        # wide groups: still per query head
         assert _decode_ws(h, 3, 8 * 40, 1000, pkv._DecodeOpts(0, 64, 0)) == _ws_expected(3, 320, 8, 16)
     finally:
         pkv.lib().kv_pool_destroy(h)

@@ -92,3 +92,20 @@ def test_prefix_plus_chunk_config():
     # and the first rows through the oracle's own multi-row chunk form
     ref = oracle.paged_prefill_chunk(opool, q[:3].cpu(), wl.BF16, paging.tables[0], P0, np.float32(d ** -0.5))
     assert max_abs_diff(out[:3], ref) <= TOL
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.05], ids=["zero", "negative"])
+def test_chunk_parity_nonpositive_scale(scale):
+    """A softmax scale <= 0 (the C-ABI takes any float): scale 0 gives uniform weights over
+    each row's keys, a negative scale favours the keys least aligned with q; causal masking
+    must still exclude the later keys."""
+    P0, C, H_q, H_kv, d = 60, 140, 16, 2, 128
+    paging, k, v, q = chunk_case(P0, C, H_q, H_kv, d, wl.BF16, 790)
+    pool = pkv.KVPool(k.to(DEV).unsqueeze(0), v.to(DEV).unsqueeze(0), wl.BF16, d,
+                      device_status=torch.zeros(1, dtype=torch.int32, device=DEV))
+    out = pkv.paged_prefill_chunk_attn(pool, 0, q.to(DEV), paging.tables[0].to(DEV), P0, scale)
+    torch.cuda.synchronize()
+    assert pkv.read_device_status(pool) == 0
+    ref = oracle.paged_prefill_chunk(oracle_pool_from_tensors(k, v, wl.BF16), q, wl.BF16, paging.tables[0], P0,
+                                     np.float32(scale))
+    assert max_abs_diff(out, ref) <= TOL
