@@ -364,7 +364,6 @@ int paged_decode_attn(pkv_pool_t pool, int layer, const void* q, int q_dtype, co
     if ((reinterpret_cast<uintptr_t>(q) & 3) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
     int engine = opts ? opts->engine : 0;
     if (engine < 0 || engine > 3) return PKV_ERR_ARG;
-    if (engine == 0) engine = 1;
     int P, parts;
     int rc = decode_partitioning(pool, num_seqs, num_q_heads, max_context_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;
@@ -466,7 +465,6 @@ int paged_decode_attn_cascade(pkv_pool_t pool, int layer, const void* q, int q_d
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15)) return PKV_ERR_ARG;
     int engine = opts ? opts->engine : 0;
     if (engine < 0 || engine > 3) return PKV_ERR_ARG;
-    if (engine == 0) engine = 1;
     int P, parts;
     int rc = cascade_partitioning(pool, num_seqs, num_q_heads, max_context_len, shared_prefix_len, opts, &P, &parts);
     if (rc != PKV_OK) return rc;

@@ -474,6 +474,7 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     p.prefix_blocks = a.part_base ? a.tok_base / kBlock : 0;
     p.window = a.window;
     p.hgroups = (a.G + 15) / 16;
+    p.num_seqs = a.B;
     p.q_bf16 = a.q_dtype == PKV_BF16;
     p.scale_log2 = a.scale * kLog2e;
     const WaitHook hook = wait_hook();
@@ -487,15 +488,23 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
             return PKV_ERR_UNSUPPORTED;
         rc = launch_decode_simt(p, a.kv_dtype, a.G, a.engine == 2, grid, s, tmk, tmv);
+    } else if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && a.engine == 0 && a.window == 0 &&
+               a.part_base == 0 && decode_tc_supported(a.d, a.G, a.kv_dtype) &&
+               (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
+        // wide groups (MQA-like): Q.K^T and P.V as tcgen05 MMAs
+        CUtensorMap tmq;
+        auto enc = tensor_map_encoder();
+        if (!enc || !make_q_map(&tmq, a.q, a.B, a.H_q, a.G, enc)) return PKV_ERR_CUDA;
+        rc = launch_decode_tc(p, a.kv_dtype, &tmq, tmk, tmv, s);
     } else if (a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) {
-        if (a.engine != 1) return PKV_ERR_UNSUPPORTED;
+        if (a.engine > 1) return PKV_ERR_UNSUPPORTED;
         const bool bf = a.kv_dtype == PKV_BF16;
         if (a.d == 128) rc = bf ? launch_mma16<128, true>(p, nht, grid, s, tmk, tmv)
                                 : launch_mma16<128, false>(p, nht, grid, s, tmk, tmv);
         else if (a.d == 64) rc = bf ? launch_mma16<64, true>(p, nht, grid, s, tmk, tmv)
                                     : launch_mma16<64, false>(p, nht, grid, s, tmk, tmv);
     } else if (is_quantized(a.kv_dtype)) {
-        if (a.engine != 1) return PKV_ERR_UNSUPPORTED;
+        if (a.engine > 1) return PKV_ERR_UNSUPPORTED;
         rc = launch_decode_quant(p, a.kv_dtype, a.d, nht, grid, s, tmk, tmv);
     }
     if (rc != PKV_OK) return rc;

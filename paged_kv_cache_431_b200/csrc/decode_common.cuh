@@ -20,6 +20,7 @@ struct DecodeParams {
     float* ws_ml;
     int32_t* status;
     int W, H_q, H_kv, G, N, part_tokens, max_parts;
+    int num_seqs;
     // Partitions cover tokens tok_base .. ctx-1 and write workspace slots part_base + part of
     // a row of `slots`.  Plain decode: 0, 0, max_parts.  Shared-prefix (cascade) decode:
     // tok_base = prefix length, part_base = key splits of the prefix (slots 0 .. part_base-1
@@ -83,6 +84,11 @@ __device__ __forceinline__ uint32_t swz128(uint32_t tile, int t, int c)
 bool decode_simt_supported(int d, int G, int kv_dtype);
 int launch_decode_simt(const DecodeParams& p, int kv_dtype, int G, bool f2, dim3 grid, cudaStream_t s,
                        const CUtensorMap* tmk, const CUtensorMap* tmv);
+
+// tcgen05 decode for groups of 64 or 128 query heads (decode_tc.cu).
+bool decode_tc_supported(int d, int G, int kv_dtype);
+int launch_decode_tc(const DecodeParams& p, int kv_dtype, const CUtensorMap* tmq, const CUtensorMap* tmk,
+                     const CUtensorMap* tmv, cudaStream_t s);
 
 // Launch the quantized-pool decode kernel (decode_quant.cu).
 int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,

@@ -60,7 +60,7 @@ struct DecodeArgs {
     float* ws_o;            // [B][H_q][max_parts][d]
     float* ws_ml;           // [B][H_q][max_parts][2]
     int32_t* status;
-    int engine;             // 1 mma, 2 fma
+    int engine;             // 0 auto, 1 warp-level mma.sync, 2 / 3 CUDA-core FMA
     int tok_base = 0;       // first token the partitions cover (cascade: the prefix length)
     int part_base = 0;      // first workspace slot they write (cascade: 1)
     int window = 0;         // sliding window (tokens a query sees), 0 = whole context

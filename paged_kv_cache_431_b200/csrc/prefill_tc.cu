@@ -27,6 +27,7 @@
 // PKV_DEV_TIMEOUT and the CTA winds down.
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace pkv {
 
@@ -62,164 +63,6 @@ struct TcParams {
     int hold_tile;          // test hook: the K copy of this CTA-local key tile is never issued (-1: none)
     long long wait_cycles;  // bound of every wait (SM cycles)
 };
-
-// ---- tcgen05 wrappers ------------------------------------------------------
-
-__device__ __forceinline__ uint64_t sdesc_k128(uint32_t addr)
-{
-    // K-major, 128-byte swizzle: rows of 128 B, 8-row atoms 1024 B apart (SBO), LBO unused (16 B)
-    return (uint64_t)((addr >> 4) & 0x3fff) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ uint64_t sdesc_mn128(uint32_t addr, uint32_t lbo_bytes)
-{
-    // MN-major, 128-byte swizzle: 64-element MN groups lbo_bytes apart (LBO), 8-row K groups
-    // 1024 B apart (SBO)
-    return (uint64_t)((addr >> 4) & 0x3fff) | ((uint64_t)((lbo_bytes >> 4) & 0x3fff) << 16) |
-           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major, int M, int N)
-{
-    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
-        : "memory");
-}
-
-// D (TMEM) += A (TMEM) . B (shared memory descriptor)
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u)
-        : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
-          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
-          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8])
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-        : "memory");
-}
-
-// Wait with a bound; on timeout record it and raise the CTA's abort flag.
-__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
-                                              long long limit)
-{
-    if (*abort_flag) return false;
-    if (mbar_wait_bounded(bar, parity, limit)) return true;
-    *abort_flag = 1;
-    flag_status(status, PKV_DEV_TIMEOUT);
-    return false;
-}
-
-// max(a, b, c) in one instruction (sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c)
-{
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction.
-__device__ __forceinline__ unsigned long long f2bits(float2 a) { return *reinterpret_cast<unsigned long long*>(&a); }
-__device__ __forceinline__ float2 bitsf2(unsigned long long d) { return *reinterpret_cast<float2*>(&d); }
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
-{
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)), "l"(f2bits(c)));
-    return bitsf2(d);
-}
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)));
-    return bitsf2(d);
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
-{
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2bits(a)), "l"(f2bits(b)));
-    return bitsf2(d);
-}
 
 struct Bars {
     uint64_t q_full;
@@ -456,7 +299,6 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         const uint32_t tO = tS + 128;
         const float sl = p.scale_log2;
         const bool pos_scale = sl > 0.f;
-        const float slx = pos_scale ? sl : 1.f;              // scale applied inside the exponent
         float m_used = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
@@ -465,66 +307,72 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 break;
             }
             tc_fence_after();
-            // the row's 128 scores of this key tile, read from TMEM once
+            // pass 1: the row maximum of the tile's 128 scores (64 at a time), in three-input
+            // maxima; the scale is applied before the causal mask, so any scale sign works
             const int key0 = (t_lo + t) * kBN;
             const bool need_mask = key0 + kBN > kmin_tile;
-            float v[kBN];
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(&v[32 * c]));
-            tmem_wait_ld();
-            if (!pos_scale) {   // a scale <= 0: apply it before the maximum (slx is then 1)
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                tmem_ld32(tS + 64 * hh, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+                tmem_wait_ld();
+                if (!pos_scale) {
 #pragma unroll
-                for (int j = 0; j < kBN; ++j) v[j] *= sl;
+                    for (int j = 0; j < 64; ++j) v[j] *= sl;
+                }
+                if (need_mask) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (key0 + 64 * hh + j >= kmax) v[j] = -INFINITY;
+                }
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[j + 2 * k], v[j + 2 * k + 1]);
             }
-            if (need_mask) {
-#pragma unroll
-                for (int j = 0; j < kBN; ++j)
-                    if (key0 + j >= kmax) v[j] = -INFINITY;
-            }
-            // row maximum: three-input maxima in four independent chains
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int j = 0; j < kBN; j += 8)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[j + 2 * k], v[j + 2 * k + 1]);
             float mx = fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], -INFINITY);
             if (pos_scale) mx *= sl;
             float m_new = m_used;
             if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
             const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
-            // P = 2^(score - m) as high + low 16-bit parts, back into the score's columns:
+            // P = 2^(scale * score - m) as high + low 16-bit parts, back into the score's columns:
             // keys 32c .. 32c+31 -> columns 32c .. 32c+15 (high), 32c+16 .. 32c+31 (low).
             // bf16: the high part is the truncation (upper half of the fp32 word), the low part
             // the truncated remainder, both by byte permutes.
+            // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
-            const float2 slx2 = make_float2(slx, slx), mref2 = make_float2(-mref, -mref);
+            const float2 sl2 = make_float2(sl, sl), mref2 = make_float2(-mref, -mref);
             float2 sum2 = make_float2(0.f, 0.f);
-            // 16 keys at a time: keys 32c + 16h .. +15 -> high parts in columns 32c + 8h .. +7,
-            // low parts in columns 32c + 16 + 8h .. +7
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                float v[32];
+                tmem_ld32(tS + 32 * c, v);
+                tmem_wait_ld();
+                uint32_t w[32];
 #pragma unroll
-            for (int c16 = 0; c16 < kBN / 16; ++c16) {
-                uint32_t wh[8], wl[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = 16 * c16 + 2 * e;
-                    const float2 a = ffma2(make_float2(v[j], v[j + 1]), slx2, mref2);
+                for (int e = 0; e < 16; ++e) {
+                    float2 a = ffma2(make_float2(v[2 * e], v[2 * e + 1]), sl2, mref2);
+                    if (need_mask) {
+                        if (key0 + 32 * c + 2 * e >= kmax) a.x = -INFINITY;
+                        if (key0 + 32 * c + 2 * e + 1 >= kmax) a.y = -INFINITY;
+                    }
                     const float2 pp = make_float2(ex2(a.x), ex2(a.y));
                     if constexpr (BF16) {
                         const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
-                        wh[e] = __byte_perm(u0, u1, 0x7632);
+                        w[e] = __byte_perm(u0, u1, 0x7632);
                         const float2 rr = fsub2(pp, make_float2(__uint_as_float(u0 & 0xffff0000u),
                                                                 __uint_as_float(u1 & 0xffff0000u)));
-                        wl[e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+                        w[16 + e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                     } else {
-                        wh[e] = pack2<false>(pp.x, pp.y);
-                        const float2 back = unpack2<false>(wh[e]);
-                        wl[e] = pack2<false>(pp.x - back.x, pp.y - back.y);
+                        w[e] = pack2<false>(pp.x, pp.y);
+                        const float2 back = unpack2<false>(w[e]);
+                        w[16 + e] = pack2<false>(pp.x - back.x, pp.y - back.y);
                     }
                     sum2 = fadd2(sum2, pp);
                 }
-                const uint32_t col = 32 * (c16 >> 1) + 8 * (c16 & 1);
-                tmem_st8u(tS + col, wh);
-                tmem_st8u(tS + col + 16, wl);
+                tmem_st32u(tS + 32 * c, w);
             }
             l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;
