@@ -18,15 +18,16 @@
 //   warp 0      TMA producer: Q once (3-D boxes over [sequence][head][dim]), then per key
 //               tile one 16-row box pair per paged block into a 2-stage K ring and V ring
 //               (128-byte swizzle, no multicast);
-//   warp 1      allocates 256 TMEM columns (S, later P: 0..63; O: 128..255) and issues
-//               every MMA from one thread;
+//   warp 1      allocates 256 TMEM columns (S, later P, of even tiles: 0..63, of odd tiles:
+//               64..127; O: 128..255) and issues every MMA from one thread, in the order
+//               QK(0), QK(1), then per tile t P.V(t), QK(t+2): the scores of tile t+1 are
+//               computed while the softmax of tile t runs;
 //   warps 2..5  softmax, one thread per query row (= TMEM lane): read the row's own 32 or
 //               64 scores, mask what lies past its partition's end, keep the running max
 //               lazily (it moves only when the new max exceeds the old by 2^8, then the
 //               thread rescales its O row), and store P as a high and a low 16-bit part
 //               over the scores (two MMAs keep P . V at ~16 mantissa bits).
-// Two CTAs fit one SM (97 KiB of shared memory, 256 TMEM columns each): while one CTA's
-// softmax runs, the other's copies and MMAs proceed.  Partials (o, m, l) of sequences longer
+// Two CTAs fit one SM (97 KiB of shared memory, 256 TMEM columns each).  Partials (o, m, l) of sequences longer
 // than one partition go to the decode workspace and are merged by decode_reduce, as in the
 // other decode engines.  Every wait is bounded; a timeout sets PKV_DEV_TIMEOUT.
 #include "decode_common.cuh"
@@ -45,7 +46,7 @@ constexpr int kQBytes = 2 * kQBox;              // 32 KiB
 constexpr int kKVBox = kBN * 128;               // one 64-dim box of a K (V) tile: 64 rows x 128 B
 constexpr int kKVBytes = 2 * kKVBox;            // 16 KiB per K (or V) stage
 constexpr int kSmem = kQBytes + kNS * 2 * kKVBytes + 1024;
-constexpr uint32_t kTmemCols = 256;             // S / P at 0, O at 128
+constexpr uint32_t kTmemCols = 256;             // S / P of even tiles at 0, of odd tiles at 64, O at 128
 constexpr int kThreads = 192;                   // producer, MMA, 4 softmax warps
 constexpr float kRescaleSlack = 8.f;            // log2 units
 
@@ -55,8 +56,9 @@ struct TcDecodeBars {
     uint64_t k_empty[kNS];
     uint64_t v_full[kNS];
     uint64_t v_empty[kNS];
-    uint64_t s_full;      // S(t) is in TMEM (every earlier MMA of the CTA is done too)
-    uint64_t p_full;      // P(t) stored by the 4 softmax warps (and V rows past an end zeroed)
+    uint64_t s_full[2];   // S(t) is in buffer t % 2 (every MMA issued before it is done too)
+    uint64_t p_full[2];   // P(t) stored by the 4 softmax warps (and V rows past an end zeroed)
+    uint64_t pv_done;     // completes once per P . V, in order
     uint64_t o_done;      // the last P . V is done
     uint64_t mma_drain;   // every MMA is done (before TMEM is freed)
 };
@@ -118,8 +120,11 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
             mbar_init(smem_u32(&bars.v_full[s]), 1);
             mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
-        mbar_init(smem_u32(&bars.s_full), 1);
-        mbar_init(smem_u32(&bars.p_full), 4);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&bars.s_full[x]), 1);
+            mbar_init(smem_u32(&bars.p_full[x]), 4);
+        }
+        mbar_init(smem_u32(&bars.pv_done), 1);
         mbar_init(smem_u32(&bars.o_done), 1);
         mbar_init(smem_u32(&bars.mma_drain), 1);
         mbar_fence_init();
@@ -210,36 +215,48 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
         if (lane == 0) {
             const uint32_t id_qk = idesc_f16(BF16, false, kM, kBN);
             const uint32_t id_pv = idesc_f16(BF16, true, kM, kD);
-            const uint32_t tS = tmem, tO = tmem + 128;
-            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status, p.wait_cycles);
-            for (int t = 0; ok && t < ntiles; ++t) {
+            const uint32_t tO = tmem + 128;
+            // S(t) = Q . K(t)^T into buffer t % 2: M 128 rows, N 64 keys, 8 steps of K = 16 dims
+            auto qk = [&](int t) -> bool {
                 const int st = t % kNS;
-                // S = Q . K^T: M 128 rows, N 64 keys, 8 steps of K = 16 dims
-                if (!wait_or_abort(smem_u32(&bars.k_full[st]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait_or_abort(smem_u32(&bars.k_full[st]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles))
+                    return false;
                 tc_fence_after();
                 const uint32_t kbase = sK + st * kKVBytes;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t qoff = (ks >> 2) * kQBox + (ks & 3) * 32;
                     const uint32_t koff = (ks >> 2) * kKVBox + (ks & 3) * 32;
-                    umma(tS, sdesc_k128(sQ + qoff), sdesc_k128(kbase + koff), id_qk, ks > 0);
+                    umma(tmem + 64 * (t & 1), sdesc_k128(sQ + qoff), sdesc_k128(kbase + koff), id_qk, ks > 0);
                 }
-                umma_commit(smem_u32(&bars.s_full));
+                umma_commit(smem_u32(&bars.s_full[t & 1]));
                 umma_commit(smem_u32(&bars.k_empty[st]));
+                return true;
+            };
+            // Tensor-core order: QK(0), QK(1), then per tile t: P.V(t), QK(t+2) -- QK(t+1) runs
+            // while the softmax of tile t does, and QK(t+2) overwrites buffer t % 2 only after
+            // P.V(t) has read it (one thread's MMAs execute in order).
+            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status, p.wait_cycles) && qk(0) &&
+                      (ntiles < 2 || qk(1));
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int st = t % kNS;
                 // O += P . V: A = P from TMEM (per 32 keys 16 columns of high parts, then 16 of
                 // low parts), B = V as an MN-major operand, 4 steps of 16 keys
-                if (!wait_or_abort(smem_u32(&bars.p_full), t & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait_or_abort(smem_u32(&bars.p_full[t & 1]), (t >> 1) & 1, &s_abort, p.status, p.wait_cycles)) break;
                 if (!wait_or_abort(smem_u32(&bars.v_full[st]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
                 tc_fence_after();
                 const uint32_t vbase = sV + st * kKVBytes;
+                const uint32_t tP = tmem + 64 * (t & 1);
 #pragma unroll
                 for (int ks = 0; ks < kBN / 16; ++ks) {
                     const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBox);
-                    const uint32_t a = tS + 32 * (ks >> 1) + 8 * (ks & 1);
+                    const uint32_t a = tP + 32 * (ks >> 1) + 8 * (ks & 1);
                     umma_ts(tO, a, bv, id_pv, !(t == 0 && ks == 0));
                     umma_ts(tO, a + 16, bv, id_pv, true);
                 }
                 umma_commit(smem_u32(&bars.v_empty[st]));
+                umma_commit(smem_u32(&bars.pv_done));
+                if (t + 2 < ntiles && !qk(t + 2)) break;
             }
             umma_commit(smem_u32(&bars.o_done));
             // every MMA this thread issued, also on an abort, is done before TMEM is freed
@@ -252,19 +269,21 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
         const int r = quarter * 32 + lane;           // query row = TMEM lane
         const int s = r / G, h = r - s * G;          // sequence of the CTA, query head in the group
         const int b = b0 + s;
-        const uint32_t tS = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t tO = tS + 128;
+        const uint32_t tL = tmem + ((uint32_t)(quarter * 32) << 16);   // this warp's lane quarter
+        const uint32_t tO = tL + 128;
         const float sl = p.scale_log2;
         const int my_end = end_s[s];
         const int my_col = s * kps;                  // this row's keys: columns my_col .. my_col + kps - 1
         float m_used = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
-            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full), t & 1, &s_abort, p.status, p.wait_cycles))) {
+            if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.s_full[t & 1]), (t >> 1) & 1, &s_abort, p.status,
+                                                        p.wait_cycles))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
+            const uint32_t tS = tL + 64 * (t & 1);   // this tile's S / P buffer
             const int key0 = tok_lo + t * kps;       // token of this row's first column
             const int nvalid = min(kps, max(0, my_end - key0));
             float v[64];
@@ -318,8 +337,16 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
             }
             l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;
-            // the running max moved: rescale this row of O (P . V(t-1) is done: s_full(t) says so)
+            // the running max moved: rescale this row of O once P . V(t-1) is done (P . V(t-2)
+            // is: QK(t) came after it, and s_full(t) covers every earlier MMA; P . V(t) waits
+            // for this tile's P)
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (!__all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.pv_done), (t - 1) & 1, &s_abort, p.status,
+                                                            p.wait_cycles))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < kD / 32; ++c) {
                     float o[32];
@@ -355,7 +382,7 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars.p_full));
+            if (lane == 0) mbar_arrive(smem_u32(&bars.p_full[t & 1]));
         }
         if (ok && __all_sync(0xffffffffu, wait_or_abort(smem_u32(&bars.o_done), 0, &s_abort, p.status, p.wait_cycles))) {
             tc_fence_after();
