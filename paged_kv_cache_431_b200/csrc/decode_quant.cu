@@ -377,17 +377,12 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             for (int c = 0; c < 4; ++c) o[mt][hn][c] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
 
-    // Tiles j0 + s, s = 0 .. STAGES-1: the inner loop is unrolled, so each copy's ring stage
-    // (and every shared-memory address derived from it) is a compile-time constant.
     int j = 0;
     bool ok = true;
-    for (int j0 = 0; ok && j0 < ntiles; j0 += STAGES) {
-#pragma unroll
-    for (int s = 0; s < STAGES; ++s) {
-        j = j0 + s;
-        if (j >= ntiles) break;
+    for (; j < ntiles; ++j) {
+        const int s = j % STAGES;
         // the whole warp gives up together (its mma.sync needs every lane)
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (j0 / STAGES) & 1, p.wait_cycles))) {
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&bars[s]), (j / STAGES) & 1, p.wait_cycles))) {
             ok = false;
             break;
         }
@@ -525,7 +520,6 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             fence_proxy_async_smem();
             issue(j + STAGES);
         }
-    }
     }
 
     if (!ok) {   // no copy may still be landing in this CTA's shared memory when it exits

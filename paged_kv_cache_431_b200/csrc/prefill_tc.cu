@@ -307,28 +307,28 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 break;
             }
             tc_fence_after();
-            // pass 1: the row maximum of the tile's 128 scores, in three-input maxima (all four
-            // TMEM loads in flight at once); the scale is applied before the causal mask, so any
-            // scale sign works
+            // pass 1: the row maximum of the tile's 128 scores (64 at a time), in three-input
+            // maxima; the scale is applied before the causal mask, so any scale sign works
             const int key0 = (t_lo + t) * kBN;
             const bool need_mask = key0 + kBN > kmin_tile;
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
-            {
-                float v[128];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(&v[32 * c]));
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                tmem_ld32(tS + 64 * hh, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(tS + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
                 tmem_wait_ld();
                 if (!pos_scale) {
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) v[j] *= sl;
+                    for (int j = 0; j < 64; ++j) v[j] *= sl;
                 }
                 if (need_mask) {
 #pragma unroll
-                    for (int j = 0; j < 128; ++j)
-                        if (key0 + j >= kmax) v[j] = -INFINITY;
+                    for (int j = 0; j < 64; ++j)
+                        if (key0 + 64 * hh + j >= kmax) v[j] = -INFINITY;
                 }
 #pragma unroll
-                for (int j = 0; j < 128; j += 8)
+                for (int j = 0; j < 64; j += 8)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) m4[k] = fmax3(m4[k], v[j + 2 * k], v[j + 2 * k + 1]);
             }
@@ -341,18 +341,15 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             // keys 32c .. 32c+31 -> columns 32c .. 32c+15 (high), 32c+16 .. 32c+31 (low).
             // bf16: the high part is the truncation (upper half of the fp32 word), the low part
             // the truncated remainder, both by byte permutes.
-            // pass 2: reread the scores 32 at a time -- chunk c+1 is loaded while chunk c is
-            // exponentiated, packed and stored over its own columns
+            // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             const float2 sl2 = make_float2(sl, sl), mref2 = make_float2(-mref, -mref);
             float2 sum2 = make_float2(0.f, 0.f);
-            float vb[2][32];
-            tmem_ld32(tS, vb[0]);
-            tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
-                if (c + 1 < kBN / 32) tmem_ld32(tS + 32 * (c + 1), vb[(c + 1) & 1]);
-                const float(&v)[32] = vb[c & 1];
+                float v[32];
+                tmem_ld32(tS + 32 * c, v);
+                tmem_wait_ld();
                 uint32_t w[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -376,7 +373,6 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                     sum2 = fadd2(sum2, pp);
                 }
                 tmem_st32u(tS + 32 * c, w);
-                if (c + 1 < kBN / 32) tmem_wait_ld();
             }
             l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;

@@ -257,7 +257,7 @@ def test_cuda_core_engines(engine, G, dtype):
 
 def test_workspace_reuse_across_shapes():
     """One workspace, never cleared by the caller, serves a series of split-K calls of
-    different shapes in stream order (each call clears its own counters)."""
+    different shapes in stream order (each call writes every partial it reads)."""
     g = wl.generator(1400)
     H_q, H_kv, d = 32, 8, 128
     cases = []
