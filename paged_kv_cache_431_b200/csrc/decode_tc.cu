@@ -15,9 +15,12 @@
 // O += P . V (M 128, N 128, K 64) takes every sequence's rows from its own keys only.  At
 // G = 64 half of the tensor work is spent on the zero blocks; the decode is bound by HBM,
 // and the tensor pipe has room for that.
-//   warp 0      TMA producer: Q once (3-D boxes over [sequence][head][dim]), then per key
-//               tile one 16-row box pair per paged block into a 2-stage K ring and V ring
-//               (128-byte swizzle, no multicast);
+//   warp 0      TMA producer of Q (once, 3-D boxes over [sequence][head][dim]) and of the
+//               2-stage K ring: per key tile one 16-row box pair per paged block (128-byte
+//               swizzle, no multicast); warp 6 does the same for the V ring, so that K
+//               tiles, freed as soon as their Q . K^T is done, are not held up behind V
+//               tiles, freed only after P . V.  The TMA row of every paged block the CTA
+//               reads is looked up once, at the start, into shared memory;
 //   warp 1      allocates 256 TMEM columns (S, later P, of even tiles: 0..63, of odd tiles:
 //               64..127; O: 128..255) and issues every MMA from one thread, in the order
 //               QK(0), QK(1), then per tile t P.V(t), QK(t+2): the scores of tile t+1 are
@@ -27,7 +30,7 @@
 //               lazily (it moves only when the new max exceeds the old by 2^8, then the
 //               thread rescales its O row), and store P as a high and a low 16-bit part
 //               over the scores (two MMAs keep P . V at ~16 mantissa bits).
-// Two CTAs fit one SM (97 KiB of shared memory, 256 TMEM columns each).  Partials (o, m, l) of sequences longer
+// Two CTAs fit one SM (99 KiB of shared memory, 256 TMEM columns each).  Partials (o, m, l) of sequences longer
 // than one partition go to the decode workspace and are merged by decode_reduce, as in the
 // other decode engines.  Every wait is bounded; a timeout sets PKV_DEV_TIMEOUT.
 #include "decode_common.cuh"
@@ -45,9 +48,11 @@ constexpr int kQBox = kM * 128;                 // one 64-dim box of Q: 128 rows
 constexpr int kQBytes = 2 * kQBox;              // 32 KiB
 constexpr int kKVBox = kBN * 128;               // one 64-dim box of a K (V) tile: 64 rows x 128 B
 constexpr int kKVBytes = 2 * kKVBox;            // 16 KiB per K (or V) stage
-constexpr int kSmem = kQBytes + kNS * 2 * kKVBytes + 1024;
+constexpr int kRowsMax = 4096 / 16;           // paged blocks of one partition (at most 4096 keys)
+constexpr int kRowsOff = kQBytes + kNS * 2 * kKVBytes;   // TMA row of every paged block of the CTA
+constexpr int kSmem = kRowsOff + 2 * kRowsMax * 4 + 1024;
 constexpr uint32_t kTmemCols = 256;             // S / P of even tiles at 0, of odd tiles at 64, O at 128
-constexpr int kThreads = 192;                   // producer, MMA, 4 softmax warps
+constexpr int kThreads = 224;                   // K producer, MMA, 4 softmax warps, V producer
 constexpr float kRescaleSlack = 8.f;            // log2 units
 
 struct TcDecodeBars {
@@ -128,6 +133,29 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
         mbar_init(smem_u32(&bars.o_done), 1);
         mbar_init(smem_u32(&bars.mma_drain), 1);
         mbar_fence_init();
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+        mbar_arrive_expect_tx(smem_u32(&bars.q_full), kQBytes);
+        tma_load_3d(sQ, &tmQ, 0, g * G, b0, smem_u32(&bars.q_full));
+        tma_load_3d(sQ + kQBox, &tmQ, 64, g * G, b0, smem_u32(&bars.q_full));
+    }
+    // TMA row of paged block kb (< 4) of tile t at rows[t * 4 + kb]: sequence kb / bps, its
+    // block kb % bps of the tile; block 0 (in bounds) past a sequence's range, where the
+    // keys are masked and the V rows zeroed
+    int* rows = reinterpret_cast<int*>(smem + kRowsOff);
+    for (int i = threadIdx.x; i < ntiles * (kBN / kBlock); i += kThreads) {
+        const int t = i >> 2, kb = i & 3;
+        const int s = kb / bps, lb = (tok_lo + t * kps) / kBlock + (kb - s * bps);
+        int blk = 0;
+        if (lb * kBlock < end_s[s]) {
+            blk = p.tables[(size_t)(b0 + s) * p.W + lb];
+            if ((unsigned)blk >= (unsigned)p.N) {
+                flag_status(p.status, PKV_DEV_BAD_BLOCK);
+                blk = 0;
+            }
+        }
+        rows[i] = (blk * p.H_kv + g) * kBlock;
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem_base)),
@@ -140,75 +168,36 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     const uint32_t tmem = s_tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        // lane kb < 4 looks up paged block kb of the tile: sequence kb / bps, its block kb % bps
-        const uint32_t qb = smem_u32(&bars.q_full);
+    if (warp == 0 || warp == 6) {
+        // ------------------------------------------------------------ producers (K: warp 0, V: warp 6)
+        const bool is_k = warp == 0;
+        uint64_t* full = is_k ? bars.k_full : bars.v_full;
+        uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+        const CUtensorMap* tm = is_k ? &tmK : &tmV;
+        const uint32_t ring = is_k ? sK : sV;
+        int issued = 0;
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-            mbar_arrive_expect_tx(qb, kQBytes);
-            tma_load_3d(sQ, &tmQ, 0, g * G, b0, qb);
-            tma_load_3d(sQ + kQBox, &tmQ, 64, g * G, b0, qb);
-        }
-        const int my_s = lane / max(1, bps), my_j = lane % max(1, bps);
-        int issued_k = 0, issued_v = 0;
-        for (int t = 0; t < ntiles; ++t) {
-            const int st = t % kNS;
-            int row = 0;
-            if (lane < kBN / kBlock) {   // 4 lanes: one paged block each
-                int blk = 0;
-                const int lb = (tok_lo + t * kps) / kBlock + my_j;   // logical block of sequence my_s
-                if (lb * kBlock < end_s[my_s]) {
-                    blk = p.tables[(size_t)(b0 + my_s) * p.W + lb];
-                    if ((unsigned)blk >= (unsigned)p.N) {
-                        flag_status(p.status, PKV_DEV_BAD_BLOCK);
-                        blk = 0;
-                    }
-                }   // past the range (or no sequence): block 0, in bounds; masked, V zeroed
-                row = (blk * p.H_kv + g) * kBlock;
-            }
-            int rows[kBN / kBlock];
-#pragma unroll
-            for (int kb = 0; kb < kBN / kBlock; ++kb) rows[kb] = __shfl_sync(0xffffffffu, row, kb);
-            bool go = true;
-            if (lane == 0 && t >= kNS)
-                go = wait_or_abort(smem_u32(&bars.k_empty[st]), ((t - kNS) / kNS) & 1, &s_abort, p.status, p.wait_cycles);
-            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
-            if (lane == 0) {
-                const uint32_t fb = smem_u32(&bars.k_full[st]);
+            for (int t = 0; t < ntiles; ++t) {
+                const int st = t % kNS;
+                if (t >= kNS &&
+                    !wait_or_abort(smem_u32(&empty[st]), ((t - kNS) / kNS) & 1, &s_abort, p.status, p.wait_cycles))
+                    break;
+                const uint32_t fb = smem_u32(&full[st]);
                 mbar_arrive_expect_tx(fb, kKVBytes);
-                if (t != p.hold_tile) {   // test hook: the withheld tile's K bytes never arrive
-#pragma unroll
-                    for (int kb = 0; kb < kBN / kBlock; ++kb)
-#pragma unroll
-                        for (int x = 0; x < 2; ++x)
-                            tma_load_2d(sK + st * kKVBytes + x * kKVBox + kb * 2048, &tmK, 64 * x, rows[kb], fb);
-                }
-            }
-            issued_k = t + 1;
-            if (lane == 0 && t >= kNS)
-                go = wait_or_abort(smem_u32(&bars.v_empty[st]), ((t - kNS) / kNS) & 1, &s_abort, p.status, p.wait_cycles);
-            if (!__shfl_sync(0xffffffffu, go ? 1 : 0, 0)) break;
-            if (lane == 0) {
-                const uint32_t fb = smem_u32(&bars.v_full[st]);
-                mbar_arrive_expect_tx(fb, kKVBytes);
+                issued = t + 1;
+                if (is_k && t == p.hold_tile) continue;   // test hook: the withheld tile's K bytes never arrive
 #pragma unroll
                 for (int kb = 0; kb < kBN / kBlock; ++kb)
 #pragma unroll
                     for (int x = 0; x < 2; ++x)
-                        tma_load_2d(sV + st * kKVBytes + x * kKVBox + kb * 2048, &tmV, 64 * x, rows[kb], fb);
+                        tma_load_2d(ring + st * kKVBytes + x * kKVBox + kb * 2048, tm, 64 * x, rows[t * 4 + kb], fb);
             }
-            issued_v = t + 1;
-        }
-        // do not leave while copies into this CTA's shared memory may be in flight
-        if (lane == 0 && s_abort) {
-            for (int t = max(0, issued_k - kNS); t < issued_k; ++t)
-                mbar_wait_bounded(smem_u32(&bars.k_full[t % kNS]), (t / kNS) & 1, p.wait_cycles);
-            for (int t = max(0, issued_v - kNS); t < issued_v; ++t)
-                mbar_wait_bounded(smem_u32(&bars.v_full[t % kNS]), (t / kNS) & 1, p.wait_cycles);
-            mbar_wait_bounded(qb, 0, p.wait_cycles);
+            // do not leave while copies into this CTA's shared memory may be in flight
+            if (s_abort) {
+                for (int t = max(0, issued - kNS); t < issued; ++t)
+                    mbar_wait_bounded(smem_u32(&full[t % kNS]), (t / kNS) & 1, p.wait_cycles);
+                if (is_k) mbar_wait_bounded(smem_u32(&bars.q_full), 0, p.wait_cycles);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
