@@ -8,15 +8,18 @@
 // Same structure as the 16-bit kernel (one warp per partition x KV head x sequence,
 // TMA ring of K/V code tiles, online softmax, split-K partials), with dequantization
 // fused into the fragment loads:
-//   * codes are converted to fp16 in registers and fed to mma.sync m16n8k16 (f16 in,
-//     fp32 accumulate); q is scaled by a power of two chosen per CTA (its largest |q|
+//   * int8 K codes go to the signed 8-bit mma.sync m16n8k32 as they are (exact int32
+//     sums), against q split into two signed 8-bit digits per element (q scaled per query
+//     head by a power of two and rounded);
+//   * the other codes are converted to fp16 in registers and fed to mma.sync m16n8k16 (f16
+//     in, fp32 accumulate); q is scaled by a power of two chosen per CTA (its largest |q|
 //     brought near 2^14, exact, undone in the score) and converted to fp16 once per warp,
 //     so a bf16 q keeps its range:
-//       - integer K codes: the code plus its offset (c + 128, c + 8) is moved into the
-//         significand of an fp16 subnormal (one byte permute or one logic op per pair,
-//         exact); the offset's share of every score, offset * sum(q), is subtracted once
-//         per score, and q is pre-scaled by a power of two so that its products with the
-//         subnormals stay well inside the accumulator's range;
+//       - int4 K codes: the code plus its offset (c + 8) is moved into the significand of
+//         an fp16 subnormal (one logic op per pair, exact); the offset's share of every
+//         score, 8 * sum(q), is subtracted once per score, and q is pre-scaled by a power
+//         of two so that its products with the subnormals stay well inside the
+//         accumulator's range;
 //       - integer V codes: the exponent trick (code + offset placed in the significand of
 //         1024.0, then 1024 + offset subtracted: exact) -- V meets the two-part P, whose
 //         low part times a subnormal loses precision in the tensor cores;
@@ -97,11 +100,10 @@ __device__ __forceinline__ void load_run(uint32_t (&w)[BYTES / 4], uint32_t tile
     }
 }
 
-// K codes become fp16 SUBNORMALS: a half whose exponent field is 0 and whose significand
-// field holds the integer u has the value u * 2^-24, exactly.  So a K code needs only to
-// be moved into the low bits of a half; the offset that makes it non-negative (u = c + 128
-// for int8, c + 8 for int4) is removed once per score (see the kernel) instead of once per
-// element.
+// int4 K codes become fp16 SUBNORMALS: a half whose exponent field is 0 and whose
+// significand field holds the integer u has the value u * 2^-24, exactly.  So a K code needs
+// only to be moved into the low bits of a half; the offset that makes it non-negative
+// (u = c + 8) is removed once per score (see the kernel) instead of once per element.
 //
 // 2^e as a float, e in [-126, 127].
 __device__ __forceinline__ float pow2f(int e)
@@ -123,13 +125,6 @@ __device__ __forceinline__ float warp_max(float v)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
-}
-
-// int8 codes, already XORed with 0x80 (u = c + 128): bytes of w picked by `sel` (nibbles
-// 0..3 pick bytes of w, 4 a zero byte) -> two halves u * 2^-24.
-__device__ __forceinline__ uint32_t u8x2(uint32_t wx, uint32_t sel)
-{
-    return __byte_perm(wx, 0u, sel);
 }
 
 // int4 codes as stored (two's complement nibbles): nibble s (0..3) of each 16-bit half
@@ -175,6 +170,16 @@ __device__ __forceinline__ uint32_t e4m3x2(uint32_t w16)
     return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
+// D += A * B, m16n8k32, signed 8-bit A (row-major, 4 regs) and B (column-major, 2 regs), int32
+// accumulate (exact).
+__device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Physical head dim that feeds MMA k-slot e (0..3: logical 2qd, 2qd+1, 2qd+8, 2qd+9)
 // of k-step ks for lane group qd.
 template <int DT, int D>
@@ -193,11 +198,8 @@ __device__ __forceinline__ int kdim(int ks, int qd, int e)
 template <int DT, int NW>
 __device__ __forceinline__ void kfrag(const uint32_t (&kw)[NW], int ks, uint32_t& b0, uint32_t& b1)
 {
-    if constexpr (DT == PKV_INT8) {
-        const uint32_t w = kw[ks] ^ 0x80808080u;
-        b0 = u8x2(w, 0x4140);
-        b1 = u8x2(w, 0x4342);
-    } else if constexpr (DT == PKV_FP8E4M3) {
+    static_assert(DT != PKV_INT8, "int8 K codes go to the 8-bit MMA unconverted");
+    if constexpr (DT == PKV_FP8E4M3) {
         b0 = e4m3x2(kw[ks]);
         b1 = e4m3x2(kw[ks] >> 16);
     } else {
@@ -252,14 +254,21 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     using Cfg = QCfg<DT, D>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int ROW = Cfg::ROW, SWZ = Cfg::SWZ;
-    // integer K codes enter Q . K^T as subnormals u * 2^-24 with u = c + OFF; odd int4
-    // nibbles enter as 16 u, and their q is pre-divided by 16.  q is pre-scaled by a power
-    // of two chosen per CTA (largest |q| brought near 2^14): for integer codes the products
-    // then stay well clear of the bottom of the accumulator's range, and for every dtype a
-    // bf16 q of any magnitude up to 2^113 fits fp16 (a bf16 q above 65504 would otherwise
-    // become inf).  The scaling is exact and is undone, with the offset, in the score.
-    constexpr bool SUBN = DT != PKV_FP8E4M3;
-    constexpr float OFF = DT == PKV_INT8 ? 128.f : 8.f;
+    // int4 K codes enter Q . K^T as subnormals u * 2^-24 with u = c + OFF; odd nibbles enter
+    // as 16 u, and their q is pre-divided by 16.  q is pre-scaled by a power of two chosen
+    // per CTA (largest |q| brought near 2^14): for int4 the products then stay well clear of
+    // the bottom of the accumulator's range, and for fp8 a bf16 q of any magnitude up to
+    // 2^113 fits fp16 (a bf16 q above 65504 would otherwise become inf).  The scaling is
+    // exact and is undone, with the offset, in the score.
+    constexpr bool SUBN = DT == PKV_INT4;
+    // int8 K codes enter Q . K^T as they are, through the signed 8-bit MMA (m16n8k32, exact
+    // int32 sums): q times 2^e_h, a power of two chosen per query head h (its largest |q|
+    // brought to [2^13, 2^14)), is rounded to an integer Q and split into two signed 8-bit
+    // digits, Q = 256 d1 + d0 with d0 in [-128, 127] and |d1| <= 64, each with its own
+    // accumulator; the score is (256 acc1 + acc0) * 2^-e_h (the int32 sum is exact).  A scale
+    // per head keeps a head with small q as precise as one with large q.
+    constexpr bool KI8 = DT == PKV_INT8;
+    constexpr float OFF = 8.f;                               // int4 code offset
     constexpr float ODD = DT == PKV_INT4 ? 0.0625f : 1.f;   // q factor on k-slots 8..15
     extern __shared__ uint8_t smem_dyn[];
     __shared__ __align__(8) uint64_t bars[STAGES];
@@ -324,12 +333,17 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
     }
 
-    // q as fp16 A fragments, k-slots assigned to physical dims by kdim(); for integer
-    // codes also -OFF * (sum of the fragments' q over d, odd int4 slots counted times 16)
-    // per head row r, r + 8: the part of 2^24 * (q . k) that the code offset adds
-    uint32_t qa[Cfg::KS][4];
+    // q as fp16 A fragments (int4, fp8), k-slots assigned to physical dims by kdim(); for
+    // int4 also -OFF * (sum of the fragments' q over d, odd slots counted times 16) per head
+    // row r, r + 8: the part of 2^24 * (q . k) that the code offset adds
+    uint32_t qa[KI8 ? 1 : Cfg::KS][4];
+    // int8: MMA k-slot (ks, half, j) of lane group qd holds head dim qd * (D/4) + 8 ks + 4 half
+    // + j, so every lane's B fragments are D/4 contiguous code bytes of a K row
+    constexpr int KS8 = D / 32;
+    uint32_t qa8[KI8 ? 2 : 1][KI8 ? KS8 : 1][4];
     float qoff[2] = {0.f, 0.f};
     int eq = 0;   // q is multiplied by 2^eq, which brings max |q| to [2^13, 2^14)
+    int eqr[2] = {0, 0};   // int8: the same per query row (rows r and r + 8)
     {
         const bool bf = p.q_bf16;
         const uint16_t* qh = static_cast<const uint16_t*>(p.q) + ((size_t)b * p.H_q + hbase) * D;
@@ -342,8 +356,47 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         for (int i = lane; i < GC * D; i += 32) qmax = fmaxf(qmax, fabsf(qv(0, i)));
         eq = pow2_shift(warp_max(qmax));
         const float qs = pow2f(eq), qo = qs * ODD;
+        if constexpr (KI8) {
+            // the largest |q| of rows r and r + 8: this lane's share of their dims, then the quad's
+            float rm[2] = {0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < Cfg::KS; ++ks) {
+            for (int ks = 0; ks < KS8; ++ks)
+#pragma unroll
+                for (int reg = 0; reg < 4; ++reg) {
+                    const int row = r + 8 * (reg & 1);
+                    const bool live = (reg & 1) ? (NHT == 2 && r + 8 < GC) : (r < GC);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        if (live) rm[reg & 1] = fmaxf(rm[reg & 1], fabsf(qv(row, qd * (D / 4) + 8 * ks + 4 * (reg >> 1) + jj)));
+                }
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                rm[hr] = fmaxf(rm[hr], __shfl_xor_sync(0xffffffffu, rm[hr], 1));
+                rm[hr] = fmaxf(rm[hr], __shfl_xor_sync(0xffffffffu, rm[hr], 2));
+                eqr[hr] = pow2_shift(rm[hr]);
+            }
+#pragma unroll
+            for (int ks = 0; ks < KS8; ++ks)
+#pragma unroll
+                for (int reg = 0; reg < 4; ++reg) {   // a0: row r, dims +0; a1: r+8, +0; a2: r, +4; a3: r+8, +4
+                    const int row = r + 8 * (reg & 1);
+                    const bool live = (reg & 1) ? (NHT == 2 && r + 8 < GC) : (r < GC);
+                    uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int Q = live ? __float2int_rn(qv(row, qd * (D / 4) + 8 * ks + 4 * (reg >> 1) + jj) *
+                                                            pow2f(eqr[reg & 1]))
+                                           : 0;
+                        const int d1 = (Q + 128) >> 8;
+                        w1 |= (uint32_t)(d1 & 0xff) << (8 * jj);
+                        w0 |= (uint32_t)((Q - 256 * d1) & 0xff) << (8 * jj);
+                    }
+                    qa8[0][ks][reg] = w0;
+                    qa8[1][ks][reg] = w1;
+                }
+        }
+#pragma unroll
+        for (int ks = 0; ks < (KI8 ? 0 : Cfg::KS); ++ks) {
             const int d0 = kdim<DT, D>(ks, qd, 0), d1 = kdim<DT, D>(ks, qd, 1);
             const int d2 = kdim<DT, D>(ks, qd, 2), d3 = kdim<DT, D>(ks, qd, 3);
             qa[ks][0] = r0 ? pack2<false>(qv(r, d0) * qs, qv(r, d1) * qs) : 0u;
@@ -365,8 +418,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             }
         }
     }
-    // log2-domain score = (acc * 2^(24-eq) + qoff) * sl for integer codes, acc * 2^-eq * sl for fp8
-    const float kq = pow2f(SUBN ? 24 - eq : -eq);
+    // log2-domain score = (acc * 2^(24-eq) + qoff) * sl for int4, acc * 2^-eq * sl for int8 / fp8
+    float kq[2];   // per query row r (hr 0) and r + 8 (hr 1)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) kq[hr] = KI8 ? pow2f(-eqr[hr]) : pow2f(SUBN ? 24 - eq : -eq);
 
     float o[Cfg::MT][NHT][4];
 #pragma unroll
@@ -404,16 +459,26 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             for (int c = 0; c < 4; ++c) sc[nt][c] = 0.f;
             uint32_t kw[Cfg::KRUN / 4];
             load_run<ROW, SWZ, Cfg::KRUN>(kw, kb, nt * 8 + r, qd * Cfg::KRUN);
+            if constexpr (KI8) {
+                int a0[4] = {0, 0, 0, 0}, a1[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int ks = 0; ks < Cfg::KS; ++ks) {
-                uint32_t b0, b1;
-                kfrag<DT>(kw, ks, b0, b1);
-                mma16816<false>(sc[nt], qa[ks], b0, b1);
+                for (int ks = 0; ks < KS8; ++ks) {
+                    mma_s8(a0, qa8[0][ks], kw[2 * ks], kw[2 * ks + 1]);
+                    mma_s8(a1, qa8[1][ks], kw[2 * ks], kw[2 * ks + 1]);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sc[nt][c] = (float)(256 * a1[c] + a0[c]);
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < Cfg::KS; ++ks) {
+                    uint32_t b0, b1;
+                    kfrag<DT>(kw, ks, b0, b1);
+                    mma16816<false>(sc[nt], qa[ks], b0, b1);
+                }
             }
         }
 
         const float sl = p.scale_log2 * sc_kv.x;
-        const float slk = sl * kq;
         float pr[2][4];
         float alpha[2];
 #pragma unroll
@@ -421,6 +486,7 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
             float x[2][2];
             float mx = -INFINITY;
             const float cb = SUBN ? qoff[hr] * sl : 0.f;
+            const float slk = sl * kq[hr];
             if (SKIP_MASK && whole) {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)

@@ -201,14 +201,19 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop (every lane waits on the same barriers, and the warp
+        // agrees on each outcome); one elected lane issues each MMA and commit.
+        {
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, wait_or_abort(bar, parity, &s_abort, p.status, p.wait_cycles));
+            };
             const uint32_t id_qk = idesc_f16(BF16, false, kM, kBN);
             const uint32_t id_pv = idesc_f16(BF16, true, kM, kD);
             const uint32_t tO = tmem + 128;
             // S(t) = Q . K(t)^T into buffer t % 2: M 128 rows, N 64 keys, 8 steps of K = 16 dims
             auto qk = [&](int t) -> bool {
                 const int st = t % kNS;
-                if (!wait_or_abort(smem_u32(&bars.k_full[st]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles))
+                if (!wait(smem_u32(&bars.k_full[st]), (t / kNS) & 1))
                     return false;
                 tc_fence_after();
                 const uint32_t kbase = sK + st * kKVBytes;
@@ -216,23 +221,23 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t qoff = (ks >> 2) * kQBox + (ks & 3) * 32;
                     const uint32_t koff = (ks >> 2) * kKVBox + (ks & 3) * 32;
-                    umma(tmem + 64 * (t & 1), sdesc_k128(sQ + qoff), sdesc_k128(kbase + koff), id_qk, ks > 0);
+                    umma_w(tmem + 64 * (t & 1), sdesc_k128(sQ + qoff), sdesc_k128(kbase + koff), id_qk, ks > 0);
                 }
-                umma_commit(smem_u32(&bars.s_full[t & 1]));
-                umma_commit(smem_u32(&bars.k_empty[st]));
+                umma_commit_w(smem_u32(&bars.s_full[t & 1]));
+                umma_commit_w(smem_u32(&bars.k_empty[st]));
                 return true;
             };
             // Tensor-core order: QK(0), QK(1), then per tile t: P.V(t), QK(t+2) -- QK(t+1) runs
             // while the softmax of tile t does, and QK(t+2) overwrites buffer t % 2 only after
             // P.V(t) has read it (one thread's MMAs execute in order).
-            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status, p.wait_cycles) && qk(0) &&
+            bool ok = wait(smem_u32(&bars.q_full), 0) && qk(0) &&
                       (ntiles < 2 || qk(1));
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int st = t % kNS;
                 // O += P . V: A = P from TMEM (per 32 keys 16 columns of high parts, then 16 of
                 // low parts), B = V as an MN-major operand, 4 steps of 16 keys
-                if (!wait_or_abort(smem_u32(&bars.p_full[t & 1]), (t >> 1) & 1, &s_abort, p.status, p.wait_cycles)) break;
-                if (!wait_or_abort(smem_u32(&bars.v_full[st]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait(smem_u32(&bars.p_full[t & 1]), (t >> 1) & 1)) break;
+                if (!wait(smem_u32(&bars.v_full[st]), (t / kNS) & 1)) break;
                 tc_fence_after();
                 const uint32_t vbase = sV + st * kKVBytes;
                 const uint32_t tP = tmem + 64 * (t & 1);
@@ -240,16 +245,16 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                 for (int ks = 0; ks < kBN / 16; ++ks) {
                     const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBox);
                     const uint32_t a = tP + 32 * (ks >> 1) + 8 * (ks & 1);
-                    umma_ts(tO, a, bv, id_pv, !(t == 0 && ks == 0));
-                    umma_ts(tO, a + 16, bv, id_pv, true);
+                    umma_ts_w(tO, a, bv, id_pv, !(t == 0 && ks == 0));
+                    umma_ts_w(tO, a + 16, bv, id_pv, true);
                 }
-                umma_commit(smem_u32(&bars.v_empty[st]));
-                umma_commit(smem_u32(&bars.pv_done));
+                umma_commit_w(smem_u32(&bars.v_empty[st]));
+                umma_commit_w(smem_u32(&bars.pv_done));
                 if (t + 2 < ntiles && !qk(t + 2)) break;
             }
-            umma_commit(smem_u32(&bars.o_done));
+            umma_commit_w(smem_u32(&bars.o_done));
             // every MMA this thread issued, also on an abort, is done before TMEM is freed
-            umma_commit(smem_u32(&bars.mma_drain));
+            umma_commit_w(smem_u32(&bars.mma_drain));
             mbar_wait_bounded(smem_u32(&bars.mma_drain), 0, p.wait_cycles);
         }
     } else {

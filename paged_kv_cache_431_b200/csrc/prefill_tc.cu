@@ -217,7 +217,9 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop (every lane waits on the same barriers); one elected
+        // lane issues each MMA and commit.
+        {
             const uint32_t id_qk = idesc_f16(BF16, false, kBM, kBN);
             const uint32_t id_pv = idesc_f16(BF16, true, kBM, kD);
             // S(x) = Q(x) . K^T of stage s: M = 128 rows, N = 128 keys, 8 steps of K = 16 dims
@@ -226,7 +228,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32;
-                    umma(tmem + 256 * x, sdesc_k128(qbase + off), sdesc_k128(kbase + off), id_qk, ks > 0);
+                    umma_w(tmem + 256 * x, sdesc_k128(qbase + off), sdesc_k128(kbase + off), id_qk, ks > 0);
                 }
             };
             // O(x) += P(x) . V of stage s: A = P from TMEM (per 32 keys: 16 columns of high
@@ -237,51 +239,54 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 for (int ks = 0; ks < kBN / 16; ++ks) {
                     const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBytes / 2);
                     const uint32_t a = tmem + 256 * x + 32 * (ks >> 1) + 8 * (ks & 1);
-                    umma_ts(tmem + 256 * x + 128, a, bv, id_pv, !(first && ks == 0));
-                    umma_ts(tmem + 256 * x + 128, a + 16, bv, id_pv, true);
+                    umma_ts_w(tmem + 256 * x + 128, a, bv, id_pv, !(first && ks == 0));
+                    umma_ts_w(tmem + 256 * x + 128, a + 16, bv, id_pv, true);
                 }
             };
-            bool ok = wait_or_abort(smem_u32(&bars.q_full), 0, &s_abort, p.status, p.wait_cycles) &&
-                      wait_or_abort(smem_u32(&bars.k_full[0]), 0, &s_abort, p.status, p.wait_cycles);
+            // every lane takes the same branch: a wait's outcome is agreed on by the warp
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, wait_or_abort(bar, parity, &s_abort, p.status, p.wait_cycles));
+            };
+            bool ok = wait(smem_u32(&bars.q_full), 0) && wait(smem_u32(&bars.k_full[0]), 0);
             if (ok) {
                 tc_fence_after();
                 qk(0, 0);
-                umma_commit(smem_u32(&bars.s_full[0]));
+                umma_commit_w(smem_u32(&bars.s_full[0]));
                 qk(1, 0);
-                umma_commit(smem_u32(&bars.s_full[1]));
-                umma_commit(smem_u32(&bars.k_empty[0]));
+                umma_commit_w(smem_u32(&bars.s_full[1]));
+                umma_commit_w(smem_u32(&bars.k_empty[0]));
             }
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int s = t % kNS, s1 = (t + 1) % kNS;
                 const bool more = t + 1 < ntiles;
                 // tile A: P . V, then its next scores
-                if (!wait_or_abort(smem_u32(&bars.p_full[0]), t & 1, &s_abort, p.status, p.wait_cycles)) break;
-                if (!wait_or_abort(smem_u32(&bars.v_full[s]), (t / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait(smem_u32(&bars.p_full[0]), t & 1)) break;
+                if (!wait(smem_u32(&bars.v_full[s]), (t / kNS) & 1)) break;
                 tc_fence_after();
                 pv(0, s, t == 0);
                 if (more) {
-                    if (!wait_or_abort(smem_u32(&bars.k_full[s1]), ((t + 1) / kNS) & 1, &s_abort, p.status, p.wait_cycles)) break;
+                    if (!wait(smem_u32(&bars.k_full[s1]), ((t + 1) / kNS) & 1)) break;
                     tc_fence_after();
                     qk(0, s1);
-                    umma_commit(smem_u32(&bars.s_full[0]));
+                    umma_commit_w(smem_u32(&bars.s_full[0]));
                 } else {
-                    umma_commit(smem_u32(&bars.o_done[0]));
+                    umma_commit_w(smem_u32(&bars.o_done[0]));
                 }
                 // tile B
-                if (!wait_or_abort(smem_u32(&bars.p_full[1]), t & 1, &s_abort, p.status, p.wait_cycles)) break;
+                if (!wait(smem_u32(&bars.p_full[1]), t & 1)) break;
                 tc_fence_after();
                 pv(1, s, t == 0);
-                umma_commit(smem_u32(&bars.v_empty[s]));
+                umma_commit_w(smem_u32(&bars.v_empty[s]));
                 if (more) {
                     qk(1, s1);
-                    umma_commit(smem_u32(&bars.s_full[1]));
-                    umma_commit(smem_u32(&bars.k_empty[s1]));
+                    umma_commit_w(smem_u32(&bars.s_full[1]));
+                    umma_commit_w(smem_u32(&bars.k_empty[s1]));
                 } else {
-                    umma_commit(smem_u32(&bars.o_done[1]));
+                    umma_commit_w(smem_u32(&bars.o_done[1]));
                 }
             }
             // Every MMA this thread issued, also on an abort, is done before TMEM is freed.
-            umma_commit(smem_u32(&bars.mma_drain));
+            umma_commit_w(smem_u32(&bars.mma_drain));
             mbar_wait_bounded(smem_u32(&bars.mma_drain), 0, p.wait_cycles);
         }
     } else {
