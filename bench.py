@@ -48,6 +48,9 @@ PROFILES = os.path.join(ROOT, "profiles")
 # the sources each kernel's DRAM-byte capture depends on (kernel, shared device code, launch setup)
 DECODE16_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                  "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
+DECODETC_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc.cu", "paged_kv_cache_431_b200/csrc/tcgen05.cuh",
+                 "paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
+                 "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 DECODEQ_SRCS = ["paged_kv_cache_431_b200/csrc/decode_quant.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                 "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
@@ -272,6 +275,9 @@ def build_decode(args, cfg, dev, rank):
     v_new = wl.normal((L, B, H_kv, d), src_dtype, gd, dev)
     out = torch.empty(L, B, H_q, d, dtype=torch.float32, device=dev)
     window = cfg.get("window", 0)
+    # paged_decode_attn's default engine takes the tcgen05 kernel for 64 or 128 query heads
+    # per KV head (16-bit pool, head dim 128, no window)
+    wide = not quant and d == 128 and H_q // H_kv in (64, 128) and not window and args.engine == 0
     ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition,
                                                           sliding_window=window), 16),
                      dtype=torch.uint8, device=dev)
@@ -358,14 +364,16 @@ def build_decode(args, cfg, dev, rank):
                        f"events); each decode "
                        f"call reads {kv / 1e9:.2f} GB of K/V"),
                 "partition_tokens": args.partition or "auto", "sliding_window": window or None,
-                "decode_engine": {0: "tensor cores (mma.sync)", 1: "tensor cores (mma.sync)",
-                                  2: "CUDA cores, packed fp32x2 FMA", 3: "CUDA cores, fp32 FMA"}[args.engine]},
+                "decode_engine": {0: "tensor cores (tcgen05)" if wide else "tensor cores (mma.sync)",
+                                  1: "tensor cores (mma.sync)", 2: "CUDA cores, packed fp32x2 FMA",
+                                  3: "CUDA cores, fp32 FMA"}[args.engine]},
         kv_bytes_per_step=kv * L, layers=L,
         seq_tokens_per_step=int((torch.clamp(ctx, max=window) if window else ctx).sum()) * L,
         roofline=dict(bound="hbm", kernel="paged_decode_attn (main + split-K merge)", alg_bytes=alg,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
-                      traffic=kernel_traffic(f"decode_{args.workload}", DECODEQ_SRCS if quant else DECODE16_SRCS)),
+                      traffic=kernel_traffic(f"decode_{args.workload}",
+                                             DECODEQ_SRCS if quant else DECODETC_SRCS if wide else DECODE16_SRCS)),
         launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",
         h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L, flush_l2=L == 1)
     return step, e2e_step, info, pool
