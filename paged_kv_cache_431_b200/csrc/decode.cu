@@ -352,16 +352,23 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
 
 // ---------------------------------------------------------------------------
 // Split-K merge: out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
-// One warp per (query head, sequence); sequences that fit one partition were written
-// directly by the main kernel and are skipped.  In the shared-prefix (cascade) form slots
-// 0 .. part_base-1 hold the prefix's partials (one per key split) and the suffix follows.
+// One warp per (query head, sequence), four heads per CTA; sequences that fit one partition
+// were written directly by the main kernel and are skipped.  In the shared-prefix (cascade)
+// form slots 0 .. part_base-1 hold the prefix's partials (one per key split) and the suffix
+// follows.  The context length (not written by the decode kernel) is read before the wait
+// for the decode grid; after it, the (m, l) pairs and up to 8 partial rows per lane go out
+// as one batch of independent loads.
 // ---------------------------------------------------------------------------
+constexpr int kMergeHeads = 4;   // warps (query heads) per merge CTA
+
 template <int D>
-__global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(32 * kMergeHeads) decode_reduce_kernel(const DecodeParams p)
 {
-    const int h = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
-    pdl_wait_primary();   // the partials of the decode kernel before this one
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.x * kMergeHeads + (threadIdx.x >> 5), b = blockIdx.y;
     const int ctx = checked_ctx(p, b, false);
+    pdl_wait_primary();   // the partials of the decode kernel before this one
+    if (h >= p.H_q) return;
     if (p.prefix_blocks > 0 && h == 0) {   // cascade: every table must start with row 0's prefix
         bool same = true;
         for (int j = lane; j < p.prefix_blocks; j += 32) same &= p.tables[(size_t)b * p.W + j] == p.tables[j];
@@ -371,30 +378,53 @@ __global__ void __launch_bounds__(32) decode_reduce_kernel(const DecodeParams p)
     if (p.part_base == 0 && nparts <= 1) return;
     const size_t base = ((size_t)b * p.H_q + h) * p.slots;
     const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + base;
-    float M = -INFINITY;
-    for (int i = lane; i < nparts; i += 32) M = fmaxf(M, ml[i].x);
-#pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int i = lane; i < nparts; i += 32) L += ex2(ml[i].x - M) * ml[i].y;
-#pragma unroll
-    for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-
     constexpr int V = D / 32;   // floats per lane
+    constexpr int kBatch = 8;   // partial rows loaded together
+    const float* po = p.ws_o + base * D + lane * V;
+
+    float M = -INFINITY, L = 0.f;
     float acc[V];
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
-    const float* po = p.ws_o + base * D + lane * V;
-#pragma unroll 4
-    for (int i = 0; i < nparts; ++i) {
-        const float w = ex2(ml[i].x - M);
-        if constexpr (V == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(po + (size_t)i * D);
-            acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-        } else {
-            const float2 v = *reinterpret_cast<const float2*>(po + (size_t)i * D);
-            acc[0] += w * v.x; acc[1] += w * v.y;
+    for (int i0 = 0; i0 < nparts; i0 += kBatch) {
+        // this batch's (m, l) (lane k < kBatch holds partial i0 + k) and o rows, all in flight at once
+        const int nb = min(kBatch, nparts - i0);
+        const float2 mlk = lane < nb ? ml[i0 + lane] : make_float2(-INFINITY, 0.f);
+        float v[kBatch][V];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            if (k < nb) {
+                if constexpr (V == 4) {
+                    const float4 t = *reinterpret_cast<const float4*>(po + (size_t)(i0 + k) * D);
+                    v[k][0] = t.x; v[k][1] = t.y; v[k][2] = t.z; v[k][3] = t.w;
+                } else {
+                    const float2 t = *reinterpret_cast<const float2*>(po + (size_t)(i0 + k) * D);
+                    v[k][0] = t.x; v[k][1] = t.y;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < V; ++e) v[k][e] = 0.f;
+            }
         }
+        float mb = mlk.x;
+#pragma unroll
+        for (int off = 4; off; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+        mb = __shfl_sync(0xffffffffu, mb, 0);             // the batch's max (lanes 0..7 hold it)
+        const float Mn = fmaxf(M, mb);                     // finite: every partial has a visible key
+        const float a = ex2(M - Mn);                       // rescale what the earlier batches summed
+        float lb = lane < nb ? ex2(mlk.x - Mn) * mlk.y : 0.f;
+#pragma unroll
+        for (int off = 4; off; off >>= 1) lb += __shfl_xor_sync(0xffffffffu, lb, off);
+        L = L * a + __shfl_sync(0xffffffffu, lb, 0);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] *= a;
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const float w = k < nb ? ex2(__shfl_sync(0xffffffffu, mlk.x, k) - Mn) : 0.f;
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] += w * v[k][e];
+        }
+        M = Mn;
     }
     const float inv = 1.f / L;
     float* out = p.out + ((size_t)b * p.H_q + h) * D + lane * V;
@@ -511,8 +541,8 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
     if (a.max_parts > 1 || a.part_base > 0) {
         // programmatic dependent launch: scheduled while the decode grid's last wave runs
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(a.H_q, a.B);
-        cfg.blockDim = dim3(32);
+        cfg.gridDim = dim3((a.H_q + kMergeHeads - 1) / kMergeHeads, a.B);
+        cfg.blockDim = dim3(32 * kMergeHeads);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = s;
         cudaLaunchAttribute attr;

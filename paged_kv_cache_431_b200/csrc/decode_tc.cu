@@ -28,8 +28,9 @@
 //   warps 2..5  softmax, one thread per query row (= TMEM lane): read the row's own 32 or
 //               64 scores, mask what lies past its partition's end, keep the running max
 //               lazily (it moves only when the new max exceeds the old by 2^8, then the
-//               thread rescales its O row), and store P as a high and a low 16-bit part
-//               over the scores (two MMAs keep P . V at ~16 mantissa bits).
+//               thread rescales its O row), and store P over the scores: for bf16 pools as
+//               a high and a low bf16 part (two MMAs keep P . V at ~16 mantissa bits), for
+//               fp16 pools as one fp16 part (11 bits, one MMA).
 // Two CTAs fit one SM (99 KiB of shared memory, 256 TMEM columns each).  Partials (o, m, l) of sequences longer
 // than one partition go to the decode workspace and are merged by decode_reduce, as in the
 // other decode engines.  Every wait is bounded; a timeout sets PKV_DEV_TIMEOUT.
@@ -234,8 +235,8 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                       (ntiles < 2 || qk(1));
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int st = t % kNS;
-                // O += P . V: A = P from TMEM (per 32 keys 16 columns of high parts, then 16 of
-                // low parts), B = V as an MN-major operand, 4 steps of 16 keys
+                // O += P . V: A = P from TMEM (per 32 keys 16 columns of high parts, then for
+                // bf16 16 of low parts), B = V as an MN-major operand, 4 steps of 16 keys
                 if (!wait(smem_u32(&bars.p_full[t & 1]), (t >> 1) & 1)) break;
                 if (!wait(smem_u32(&bars.v_full[st]), (t / kNS) & 1)) break;
                 tc_fence_after();
@@ -246,7 +247,7 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                     const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBox);
                     const uint32_t a = tP + 32 * (ks >> 1) + 8 * (ks & 1);
                     umma_ts_w(tO, a, bv, id_pv, !(t == 0 && ks == 0));
-                    umma_ts_w(tO, a + 16, bv, id_pv, true);
+                    if constexpr (BF16) umma_ts_w(tO, a + 16, bv, id_pv, true);   // low part
                 }
                 umma_commit_w(smem_u32(&bars.v_empty[st]));
                 umma_commit_w(smem_u32(&bars.pv_done));
@@ -299,7 +300,7 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             float2 sum2 = make_float2(0.f, 0.f);
             // P for the row's own keys, 32 at a time: columns 32c .. 32c+15 high parts,
-            // 32c+16 .. 32c+31 low parts; the other sequence's columns get zeros
+            // 32c+16 .. 32c+31 low parts (bf16); the other sequence's columns get zeros
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 if (32 * c >= kps) break;
@@ -314,14 +315,13 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                         const float2 rr = fsub2(pp, make_float2(__uint_as_float(u0 & 0xffff0000u),
                                                                 __uint_as_float(u1 & 0xffff0000u)));
                         w[16 + e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
-                    } else {
+                    } else {   // fp16 P in one part: 11 bits, relative error <= 2^-12
                         w[e] = pack2<false>(pp.x, pp.y);
-                        const float2 back = unpack2<false>(w[e]);
-                        w[16 + e] = pack2<false>(pp.x - back.x, pp.y - back.y);
                     }
                     sum2 = fadd2(sum2, pp);
                 }
-                tmem_st32u(tS + my_col + 32 * c, w);
+                if constexpr (BF16) tmem_st32u(tS + my_col + 32 * c, w);
+                else tmem_st16u(tS + my_col + 32 * c, *reinterpret_cast<const uint32_t(*)[16]>(&w[0]));
             }
             if (kps == 32) {   // two sequences: zero P over the other one's keys
                 uint32_t z[32];

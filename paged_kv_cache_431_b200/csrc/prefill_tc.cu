@@ -17,8 +17,9 @@
 //               lane): read the row's 128 scores, mask (causal bound, window, end of
 //               sequence), keep the running max lazily (it moves only when the new max
 //               exceeds the old by 2^8, then O is rescaled in TMEM), and write P back into
-//               the score's own TMEM columns as a high and a low 16-bit part (two MMAs keep
-//               P . V at ~16 mantissa bits), where the P . V MMA reads it as its A operand.
+//               the score's own TMEM columns, where the P . V MMA reads it as its A operand:
+//               for bf16 pools as a high and a low bf16 part (two MMAs keep P . V at ~16
+//               mantissa bits), for fp16 pools as one fp16 part (11 bits, one MMA).
 // The two tiles ping-pong: while the softmax warps of one tile work, the tensor cores run
 // the other tile's P . V and next Q.K^T, so neither unit waits for the other:
 //   MMA order per key tile t:  P.V(A, t), Q.K^T(A, t+1), P.V(B, t), Q.K^T(B, t+1).
@@ -232,7 +233,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                 }
             };
             // O(x) += P(x) . V of stage s: A = P from TMEM (per 32 keys: 16 columns of high
-            // parts, then 16 of low parts), B = V as an MN-major operand; 8 steps of 16 keys
+            // parts, then for bf16 16 of low parts), B = V as an MN-major operand; 8 steps of 16 keys
             auto pv = [&](int x, int s, bool first) {
                 const uint32_t vbase = sV + s * kKVBytes;
 #pragma unroll
@@ -240,7 +241,7 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                     const uint64_t bv = sdesc_mn128(vbase + ks * 2048, kKVBytes / 2);
                     const uint32_t a = tmem + 256 * x + 32 * (ks >> 1) + 8 * (ks & 1);
                     umma_ts_w(tmem + 256 * x + 128, a, bv, id_pv, !(first && ks == 0));
-                    umma_ts_w(tmem + 256 * x + 128, a + 16, bv, id_pv, true);
+                    if constexpr (BF16) umma_ts_w(tmem + 256 * x + 128, a + 16, bv, id_pv, true);   // low part
                 }
             };
             // every lane takes the same branch: a wait's outcome is agreed on by the warp
@@ -342,10 +343,10 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
             float m_new = m_used;
             if (mx > m_used + kRescaleSlack || m_used == -INFINITY) m_new = mx;
             const float alpha = m_used == -INFINITY ? 0.f : ex2(m_used - m_new);
-            // P = 2^(scale * score - m) as high + low 16-bit parts, back into the score's columns:
-            // keys 32c .. 32c+31 -> columns 32c .. 32c+15 (high), 32c+16 .. 32c+31 (low).
+            // P = 2^(scale * score - m), back into the score's columns: keys 32c .. 32c+31 ->
+            // columns 32c .. 32c+15 (high part), 32c+16 .. 32c+31 (bf16 only: low part).
             // bf16: the high part is the truncation (upper half of the fp32 word), the low part
-            // the truncated remainder, both by byte permutes.
+            // the truncated remainder, both by byte permutes; fp16: P rounded to fp16.
             // pass 2: reread each 32-key chunk, exponentiate, pack, store over the same columns
             const float mref = m_new == -INFINITY ? 0.f : m_new;
             const float2 sl2 = make_float2(sl, sl), mref2 = make_float2(-mref, -mref);
@@ -370,14 +371,13 @@ prefill_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tmQ, con
                         const float2 rr = fsub2(pp, make_float2(__uint_as_float(u0 & 0xffff0000u),
                                                                 __uint_as_float(u1 & 0xffff0000u)));
                         w[16 + e] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
-                    } else {
+                    } else {   // fp16 P in one part: 11 bits, relative error <= 2^-12
                         w[e] = pack2<false>(pp.x, pp.y);
-                        const float2 back = unpack2<false>(w[e]);
-                        w[16 + e] = pack2<false>(pp.x - back.x, pp.y - back.y);
                     }
                     sum2 = fadd2(sum2, pp);
                 }
-                tmem_st32u(tS + 32 * c, w);
+                if constexpr (BF16) tmem_st32u(tS + 32 * c, w);
+                else tmem_st16u(tS + 32 * c, *reinterpret_cast<const uint32_t(*)[16]>(&w[0]));
             }
             l_run = l_run * alpha + (sum2.x + sum2.y);
             m_used = m_new;
