@@ -100,17 +100,20 @@ int layer_maps(pkv_pool* pool, int layer, const CUtensorMap** tmk, const CUtenso
     return PKV_OK;
 }
 
-// Split-K partition size: about 256 KiB of K + V per partition whatever the storage
-// dtype (512 tokens for bf16 at head_dim 128, 1024 for int8 / fp8, 2048 for int4), so the
-// partials stay near 1.6% of the bytes read; smaller (down to 128 tokens) when the batch
-// is too small to fill the GPU with one-warp CTAs.
-static int choose_partition(int B, int ctas, int max_ctx, int row_bytes, const pkv_decode_opts* o)
+// Split-K partition size: about 256 KiB of K + V per partition for 16-bit pools (512 tokens
+// at head_dim 128) and 192 KiB for quantized ones (768 tokens for int8 / fp8, 1536 for int4),
+// so the partials stay near 1.6-2% of the bytes read; smaller (halved, down to 128 or 192
+// tokens) when the batch is too small to fill the GPU with one-warp CTAs.  The quantized
+// sizes were measured on the long-context layer: 768 against 1024 tokens took int8 from 495
+// to 475 us per call and fp8 from 618 to 586, 1536 against 2048 took int4 from 560 to 524
+// (partitions of 3 * 2^k tokens beat the powers of two on both sides of them).
+static int choose_partition(int B, int ctas, int max_ctx, int row_bytes, bool quantized, const pkv_decode_opts* o)
 {
     if (o && o->partition_tokens > 0) return o->partition_tokens;
-    int P = 256 * 1024 / (2 * row_bytes);
+    int P = (quantized ? 192 : 256) * 1024 / (2 * row_bytes);
     P = P < 128 ? 128 : (P > 4096 ? 4096 : P);
     const long target = 4L * num_sms() * 8;
-    while (P > 128) {
+    while (P >= 256) {   // halves down to 128 (powers of two) or 192 (3 * 2^k) tokens
         const long parts = (max_ctx + P - 1) / P;
         if ((long)B * ctas * (parts > 0 ? parts : 1) >= target) break;
         P /= 2;
@@ -322,7 +325,8 @@ static int decode_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, i
     if (window < 0) return PKV_ERR_ARG;
     // with a window a sequence's partitions start at the block holding ctx - window
     const int span = (window > 0 && max_ctx > window + PKV_BLOCK_SIZE - 1) ? window + PKV_BLOCK_SIZE - 1 : max_ctx;
-    *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), span, pool->row_bytes, opts);
+    *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), span, pool->row_bytes,
+                          is_quantized(pool->d.kv_dtype), opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
     *max_parts = span > 0 ? (span + *P - 1) / *P : 1;
     return PKV_OK;
@@ -418,7 +422,7 @@ static int cascade_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, 
 {
     const int rest = max_ctx - prefix_len;
     *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), rest > 0 ? rest : 1, pool->row_bytes,
-                          opts);
+                          is_quantized(pool->d.kv_dtype), opts);
     if (!valid_partition(*P)) return PKV_ERR_ARG;
     *suffix_parts = rest > 0 ? (rest + *P - 1) / *P : 1;
     return PKV_OK;

@@ -184,12 +184,12 @@ def _ws_expected(B, H_q, H_kv, parts, d=128):
     return B * H_q * parts * (d + 2) * 4
 
 
-@pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 1024), (pkv.FP8E4M3, 1024),
-                                     (pkv.INT4, 2048)])
+@pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 768), (pkv.FP8E4M3, 768),
+                                     (pkv.INT4, 1536)])
 def test_decode_workspace_follows_the_partition_policy(dtype, P):
-    """Split-K partitions of ~256 KiB of K + V whatever the storage dtype (512 / 1024 / 2048 tokens at
-    d = 128) when the batch fills the GPU; the workspace is fp32 o[d] + (m, l) per (sequence, query
-    head, partition)."""
+    """Split-K partitions of ~256 KiB of K + V for 16-bit pools and ~192 KiB for quantized ones (512 /
+    768 / 1536 tokens at d = 128) when the batch fills the GPU; the workspace is fp32 o[d] + (m, l)
+    per (sequence, query head, partition)."""
     kw = dict(num_kv_heads=8, head_dim=128, kv_dtype=dtype)
     if dtype in pkv.QUANTIZED:
         kw.update(k_scale=0x30000, v_scale=0x40000)
@@ -199,7 +199,7 @@ def test_decode_workspace_follows_the_partition_policy(dtype, P):
         B, H_q, ctx = 170, 64, 8192
         assert _decode_ws(h, B, H_q, ctx) == _ws_expected(B, H_q, 8, -(-ctx // P))
         # a context of one default partition: with only B * H_kv CTAs the grid cannot fill the GPU, so
-        # partitions are halved (to 128 tokens at least) and the partials come back
+        # partitions are halved (to 128 or 192 tokens at least) and the partials come back
         short = _decode_ws(h, B, H_q, P) - _ws_expected(B, H_q, 8, 2) + B * H_q * 2 * (128 + 2) * 4
         parts, rem = divmod(short, B * H_q * (128 + 2) * 4)
         assert rem == 0 and 2 <= parts <= P // 128 and parts & (parts - 1) == 0
