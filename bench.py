@@ -136,6 +136,11 @@ def source_hash(src_files):
     return h.hexdigest()
 
 
+def scaled(v, f):
+    """v * f rounded to an integer, None stays None (traffic records are per full launch)."""
+    return None if v is None else int(round(v * f))
+
+
 def kernel_traffic(key: str, src_files):
     """DRAM bytes per launch from a committed ncu summary, used only while the kernel
     sources still hash to the version that was captured."""
@@ -491,7 +496,7 @@ def build_blocks(args, cfg, dev, rank):
     back in (preemption).  Block = all layers' K and V tiles of its 8 KV heads (5.24 MB)."""
     from paged_kv_cache_431_b200 import pkv
 
-    L, H_kv, d, N = cfg["layers"], cfg["H_kv"], cfg["d"], cfg["pool_blocks"]
+    L, H_kv, d, N = args.layers or cfg["layers"], cfg["H_kv"], cfg["d"], cfg["pool_blocks"]
     n_copy, n_swap = cfg["copies"], cfg["swaps"]
     gd = wl.generator(431 + 500 + rank, dev)
     k_pool = torch.empty(L, N, H_kv, 16, d, dtype=torch.bfloat16, device=dev)
@@ -540,7 +545,8 @@ def build_blocks(args, cfg, dev, rank):
     swapped = n_swap * per_block
     peaks, kind = measured_peaks()
     info = dict(
-        config={"workload": args.workload, "description": cfg["desc"], "layers": L, "kv_heads": H_kv, "head_dim": d,
+        config={"workload": args.workload if L == cfg["layers"] else f"{args.workload} ({L} layers)",
+                "description": cfg["desc"], "layers": L, "kv_heads": H_kv, "head_dim": d,
                 "kv_dtype": "bf16", "pool_blocks_per_layer": N, "copy_pairs": n_copy, "swapped_blocks": n_swap,
                 "bytes_per_block": per_block, "parallelism": "replicas",
                 "l2": f"inputs larger than L2: each copy call moves {copied / 1e9:.2f} GB"},
@@ -548,7 +554,8 @@ def build_blocks(args, cfg, dev, rank):
         roofline=dict(bound="hbm", kernel="kv_copy_blocks", alg_bytes=2 * copied, call_index=0,
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs; a copy reads and writes each byte)",
-                      traffic=kernel_traffic("copy_blocks", BLOCKS_SRCS), swap_bytes=swapped),
+                      traffic=scaled(kernel_traffic("copy_blocks", BLOCKS_SRCS), L / cfg["layers"]),
+                      swap_bytes=swapped),
         launches_per_step=3, dtype="u8", h2d=h_ids.numel() * 4 + swapped, d2h=swapped, calls_per_step=3)
     return step, e2e_step, info, pool
 
@@ -1028,6 +1035,8 @@ def main():
                     help="--impl reference: host threads calling the oracle concurrently, one sequence "
                          "each per step (0: every usable core, at most 64; 1: one thread)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="blocks: layers of the pool (default 80); fewer for counter captures on a small pool")
     ap.add_argument("--partition", type=int, default=0,
                     help="split-K partition size in tokens (0: chosen by the library)")
     ap.add_argument("--decode-form", default="cascade", choices=["cascade", "plain"],
