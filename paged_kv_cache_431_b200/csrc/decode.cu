@@ -116,10 +116,18 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         const int row = (tbl[j] * p.H_kv + g) * kBlock;
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
         if (j == p.hold_tile) return;   // test hook: the stage's bytes never arrive
+        if constexpr (kHintKV) {   // the K/V stream is read once: first out of L2
+            const uint64_t pol = l2_evict_first();
 #pragma unroll
-        for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + x * 2048, &tmK, x * 64, row, bar);
+            for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d_hint(kdst + x * 2048, &tmK, x * 64, row, bar, pol);
 #pragma unroll
-        for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + Cfg::TILE + x * 2048, &tmV, x * 64, row, bar);
+            for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d_hint(kdst + Cfg::TILE + x * 2048, &tmV, x * 64, row, bar, pol);
+        } else {
+#pragma unroll
+            for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + x * 2048, &tmK, x * 64, row, bar);
+#pragma unroll
+            for (int x = 0; x < Cfg::NBOX; ++x) tma_load_2d(kdst + Cfg::TILE + x * 2048, &tmV, x * 64, row, bar);
+        }
     };
     if (threadIdx.x == 0) {
         for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
@@ -335,7 +343,9 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
         for (int i = lane; i < GC * (D / 4); i += 32) {
             const int h = i / (D / 4), c4 = i % (D / 4);
             const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
-            *reinterpret_cast<float4*>(p.ws_o + ws_slot(p, row0 + h, part) * D + 4 * c4) = v;
+            float4* dst = reinterpret_cast<float4*>(p.ws_o + ws_slot(p, row0 + h, part) * D + 4 * c4);
+            if constexpr (kHintPartials) st_hint(dst, v, l2_evict_last());   // the merge reads it back soon
+            else *dst = v;
         }
         if (qd == 0) {
 #pragma unroll
@@ -343,7 +353,9 @@ decode_mma16_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm
                 const int h = r + 8 * hr;
                 if (h < GC) {
                     float2 ml = make_float2(m_run[hr], l_run[hr]);
-                    *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) = ml;
+                    float2* dst = reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2);
+                    if constexpr (kHintPartials) st_hint(dst, ml, l2_evict_last());
+                    else *dst = ml;
                 }
             }
         }

@@ -9,6 +9,14 @@ namespace pkv {
 constexpr int kMaxPartTiles = 256;   // partition_tokens <= 4096
 constexpr float kLog2e = 1.4426950408889634f;
 
+// L2 cache hints of the decode kernels: the K/V stream is read once (evict_first), the
+// split-K partials are read back by the merge soon after (evict_last).
+#ifndef PKV_L2_HINTS
+#define PKV_L2_HINTS 3
+#endif
+constexpr bool kHintKV = (PKV_L2_HINTS & 1) != 0;
+constexpr bool kHintPartials = (PKV_L2_HINTS & 2) != 0;
+
 struct DecodeParams {
     const void* q;
     const int32_t* tables;

@@ -268,6 +268,10 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
     // accumulator; the score is (256 acc1 + acc0) * 2^-e_h (the int32 sum is exact).  A scale
     // per head keeps a head with small q as precise as one with large q.
     constexpr bool KI8 = DT == PKV_INT8;
+    // L2 hints (evict_first on the K/V stream, evict_last on the partials): measured faster for
+    // int8 (475 -> 468 us per long-context call) and equal for fp8, but slower for int4 (527 ->
+    // 549 us), which keeps the default policy
+    constexpr bool HINT = kHintKV && DT != PKV_INT4, HINTP = kHintPartials && DT != PKV_INT4;
     constexpr float OFF = 8.f;                               // int4 code offset
     constexpr float ODD = DT == PKV_INT4 ? 0.0625f : 1.f;   // q factor on k-slots 8..15
     extern __shared__ uint8_t smem_dyn[];
@@ -326,8 +330,14 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const int row = (tbl[j] * p.H_kv + g) * kBlock;
         mbar_arrive_expect_tx(bar, Cfg::STAGE);
         if (j == p.hold_tile) return;   // test hook: the stage's bytes never arrive
-        tma_load_2d(kdst, &tmK, 0, row, bar);
-        tma_load_2d(kdst + Cfg::TILE, &tmV, 0, row, bar);
+        if constexpr (HINT) {   // the K/V stream is read once: first out of L2
+            const uint64_t pol = l2_evict_first();
+            tma_load_2d_hint(kdst, &tmK, 0, row, bar, pol);
+            tma_load_2d_hint(kdst + Cfg::TILE, &tmV, 0, row, bar, pol);
+        } else {
+            tma_load_2d(kdst, &tmK, 0, row, bar);
+            tma_load_2d(kdst + Cfg::TILE, &tmV, 0, row, bar);
+        }
     };
     if (lane == 0) {
         for (int j = 0; j < min(STAGES, ntiles); ++j) issue(j);
@@ -628,15 +638,19 @@ decode_mmaq_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK
         const int h = i / (D / 4), c4 = i % (D / 4);
         const float4 v = *reinterpret_cast<const float4*>(&so[h * SR + 4 * c4]);
         const size_t off = final_out ? (row0 + h) * D : ws_slot(p, row0 + h, part) * D;
-        *reinterpret_cast<float4*>(dst + off + 4 * c4) = v;
+        float4* at = reinterpret_cast<float4*>(dst + off + 4 * c4);
+        if (HINTP && !final_out) st_hint(at, v, l2_evict_last());   // the merge reads it back soon
+        else *at = v;
     }
     if (!final_out && qd == 0) {
 #pragma unroll
         for (int hr = 0; hr < NHT; ++hr) {
             const int h = r + 8 * hr;
-            if (h < GC)
-                *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2) =
-                    make_float2(m_run[hr], l_run[hr]);
+            if (h < GC) {
+                float2* at = reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, row0 + h, part) * 2);
+                if (HINTP) st_hint(at, make_float2(m_run[hr], l_run[hr]), l2_evict_last());
+                else *at = make_float2(m_run[hr], l_run[hr]);
+            }
         }
     }
 }

@@ -190,8 +190,13 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
                 for (int kb = 0; kb < kBN / kBlock; ++kb)
 #pragma unroll
-                    for (int x = 0; x < 2; ++x)
-                        tma_load_2d(ring + st * kKVBytes + x * kKVBox + kb * 2048, tm, 64 * x, rows[t * 4 + kb], fb);
+                    for (int x = 0; x < 2; ++x) {
+                        if constexpr (kHintKV)
+                            tma_load_2d_hint(ring + st * kKVBytes + x * kKVBox + kb * 2048, tm, 64 * x, rows[t * 4 + kb],
+                                             fb, l2_evict_first());
+                        else
+                            tma_load_2d(ring + st * kKVBytes + x * kKVBox + kb * 2048, tm, 64 * x, rows[t * 4 + kb], fb);
+                    }
             }
             // do not leave while copies into this CTA's shared memory may be in flight
             if (s_abort) {
@@ -386,7 +391,12 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
             const size_t qrow = (size_t)b * p.H_q + (size_t)g * G + h;
             float* orow = final_out ? p.out + qrow * kD : p.ws_o + ws_slot(p, qrow, part) * kD;
             const float inv = final_out ? 1.f / l_run : 1.f;
-            if (has && !final_out) *reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, qrow, part) * 2) = make_float2(m_used, l_run);
+            const uint64_t pol = l2_evict_last();   // partials: the merge reads them back soon
+            if (has && !final_out) {
+                float2* dst = reinterpret_cast<float2*>(p.ws_ml + ws_slot(p, qrow, part) * 2);
+                if (kHintPartials) st_hint(dst, make_float2(m_used, l_run), pol);
+                else *dst = make_float2(m_used, l_run);
+            }
 #pragma unroll 1
             for (int c = 0; c < kD / 32; ++c) {
                 float o[32];
@@ -394,9 +404,12 @@ decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmQ,
                 tmem_wait_ld();
                 if (has) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(orow + 32 * c + i) =
-                            make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+                    for (int i = 0; i < 32; i += 4) {
+                        float4* dst = reinterpret_cast<float4*>(orow + 32 * c + i);
+                        const float4 v = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+                        if (kHintPartials && !final_out) st_hint(dst, v, pol);
+                        else *dst = v;
+                    }
                 }
             }
         }
