@@ -224,10 +224,12 @@ def decode_bytes(ctx_lens, B, H_q, H_kv, d, dt, window=0):
 # ------------------------------------------------------------- GPU arm --
 
 class Timed:
-    """Device timing of the K steps plus per-call events around the dominant calls."""
+    """Device timing of the K steps plus per-call events around the dominant calls.  With
+    `external`, the events can be recorded inside a CUDA-graph capture: they become event-record
+    nodes that take their timestamps at every replay."""
 
-    def __init__(self, steps, per_step):
-        mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    def __init__(self, steps, per_step, external=False):
+        mk = lambda: torch.cuda.Event(enable_timing=True, external=external)  # noqa: E731
         self.ev = [[(mk(), mk()) for _ in range(per_step)] for _ in range(steps)]
 
     def call_ms(self):
@@ -295,11 +297,11 @@ def build_decode(args, cfg, dev, rank):
             lp = l % L_phys
             pkv.kv_append(pool, lp, k_new[l], v_new[l], slots, workspace=aws)
             if ev is not None:
-                ev[l][0].record(stream)
+                ev[l][0].record()
             pkv.paged_decode_attn(pool, lp, q[l], tables, ctx_d, scale, max_ctx, out=out[l], workspace=ws,
                                   engine=args.engine, partition_tokens=args.partition, sliding_window=window)
             if ev is not None:
-                ev[l][1].record(stream)
+                ev[l][1].record()
 
     kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt, window)
     # this library's kernels per layer: the append (3 for quantized pools), the decode and, when a
@@ -434,16 +436,16 @@ def build_prefix_chunk(args, cfg, dev, rank):
     def step(ev=None):
         pkv.kv_append(pool, 0, k_dec, v_dec, dec_slots)
         if ev is not None:
-            ev[0][0].record(stream)
+            ev[0][0].record()
         decode(q_dec, out_dec)
         if ev is not None:
-            ev[0][1].record(stream)
+            ev[0][1].record()
         pkv.kv_append(pool, 0, k_chunk, v_chunk, chunk_slots)
         if ev is not None:
-            ev[1][0].record(stream)
+            ev[1][0].record()
         pkv.paged_prefill_chunk_attn(pool, 0, q_chunk, chunk_table, P0, scale, out=out_chunk)
         if ev is not None:
-            ev[1][1].record(stream)
+            ev[1][1].record()
 
     dec_kv, dec_alg = decode_bytes(ctx, B, H_q, H_kv, d, wl.BF16)
     pairs = sum(P0 + i + 1 for i in range(C))                      # causal (query, key) pairs per head
@@ -518,18 +520,18 @@ def build_blocks(args, cfg, dev, rank):
 
     def step(ev=None):
         if ev is not None:
-            ev[0][0].record(stream)
+            ev[0][0].record()
         pkv.kv_copy_blocks(pool, d_src, d_dst)
         if ev is not None:
-            ev[0][1].record(stream)
-            ev[1][0].record(stream)
+            ev[0][1].record()
+            ev[1][0].record()
         pkv.kv_swap_out(pool, d_out, host)
         if ev is not None:
-            ev[1][1].record(stream)
-            ev[2][0].record(stream)
+            ev[1][1].record()
+            ev[2][0].record()
         pkv.kv_swap_in(pool, d_in, host)
         if ev is not None:
-            ev[2][1].record(stream)
+            ev[2][1].record()
 
     # end to end: the block ids come from pinned host memory every step
     h_ids = torch.cat([src, dst, out_ids, in_ids]).pin_memory()
@@ -643,13 +645,19 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     if pkv.read_device_status(pool):
         raise RuntimeError("device status set during warm-up")
-    graph = None
-    if args.graph:   # the whole step (every layer's append and attention) as one CUDA graph
+    graph = tgraph = None
+    gtimed = Timed(1, info["calls_per_step"], external=True)
+    if args.graph:   # the whole step (every layer's append and attention) as one CUDA graph; a
+        # second capture adds event nodes around the dominant calls, for their durations only
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step()
+        tgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tgraph):
+            step(gtimed.ev[0])
         for _ in range(args.warmup):
             graph.replay()
+            tgraph.replay()
         torch.cuda.synchronize(dev)
 
     # single-layer decode workloads re-read inputs that could still sit in L2 from the step
@@ -658,16 +666,31 @@ def run_gpu(args):
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    # per-call durations (the roofline) from eager steps with events around each call
+    # per-call durations (the roofline): events around each call of eager steps; with a graph,
+    # also the event nodes of a second, evented capture of the step (one replay at a time, read
+    # after each), reported beside them
     eager_ms, timed = time_steps(step, args.steps, info["calls_per_step"], dev, world, flush)
+    call_ms = timed.call_ms()
+    graph_call_ms = None
     elapsed_ms = eager_ms
     if graph is not None:
         elapsed_ms, _ = time_steps(lambda ev=None: graph.replay(), args.steps, 1, dev, world, flush)
+        graph_call_ms = []
+        for _ in range(args.steps):
+            if flush is not None:
+                flush()
+            tgraph.replay()
+            torch.cuda.synchronize(dev)
+            graph_call_ms += gtimed.call_ms()
     clk = clocks.stop()
     if pkv.read_device_status(pool):
         raise RuntimeError("device status set during timing")
     info["config"]["step_timing"] = ("CUDA-graph replays of one captured step" if graph is not None
                                      else "eager launches") + f"; eager steps {eager_ms / args.steps:.4f} ms"
+    info["config"]["call_timing"] = ("events around each call of eager steps; graph_launch_us: event nodes "
+                                     "around each call in a second, evented capture of the step (the graph "
+                                     "timed for `value` has none)" if graph is not None
+                                     else "events around each call of eager steps")
 
     # end to end through the same calls with host buffers
     for _ in range(max(1, args.warmup)):
@@ -678,7 +701,6 @@ def run_gpu(args):
     ms_per_step = elapsed_ms / args.steps
     value = job_throughput(info["kv_bytes_per_step"], args.steps, world, elapsed_ms) / 1e9
     e2e_value = job_throughput(info["kv_bytes_per_step"], args.steps, world, e2e_ms) / 1e9
-    call_ms = timed.call_ms()
     rf = info["roofline"]
     if rf["bound"] == "hbm":
         cpk = info["calls_per_step"]
@@ -689,6 +711,9 @@ def run_gpu(args):
                     "unit": "GB/s", "frac": round(achieved / rf["peak"], 4), "peak_source": rf["peak_source"],
                     "traffic": rf["traffic"], "algorithmic_bytes_per_launch": rf["alg_bytes"],
                     "avg_launch_us": round(avg_s * 1e6, 2)}
+        if graph_call_ms:
+            gsel = graph_call_ms if "call_index" not in rf else graph_call_ms[rf["call_index"]::cpk]
+            roofline["graph_launch_us"] = round(statistics.mean(gsel) * 1e3, 2)
         if "swap_bytes" in rf:   # host-link moves: swap-out then swap-in calls
             for name, i in (("swap_out_gbs", 1), ("swap_in_gbs", 2)):
                 roofline[name] = round(rf["swap_bytes"] / (statistics.mean(call_ms[i::cpk]) * 1e-3) / 1e9, 2)
@@ -705,6 +730,8 @@ def run_gpu(args):
                     "avg_launch_us": round(avg_s * 1e6, 2),
                     "decode_call_us": round(dec_s * 1e6, 2),
                     "decode_logical_gbs": round(rf["decode_alg_bytes"] / dec_s / 1e9, 1)}
+        if graph_call_ms:
+            roofline["graph_launch_us"] = round(statistics.mean(graph_call_ms[ci::info["calls_per_step"]]) * 1e3, 2)
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
