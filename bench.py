@@ -51,6 +51,9 @@ DECODE16_SRCS = ["paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b
 DECODETC_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc.cu", "paged_kv_cache_431_b200/csrc/tcgen05.cuh",
                  "paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                  "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
+DECODETCK_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc_keys.cu", "paged_kv_cache_431_b200/csrc/tcgen05.cuh",
+                  "paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
+                  "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 DECODEQ_SRCS = ["paged_kv_cache_431_b200/csrc/decode_quant.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                 "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
@@ -285,6 +288,7 @@ def build_decode(args, cfg, dev, rank):
     # paged_decode_attn's default engine takes the tcgen05 kernel for 64 or 128 query heads
     # per KV head (16-bit pool, head dim 128, no window)
     wide = not quant and d == 128 and H_q // H_kv in (64, 128) and not window and args.engine == 0
+    keys_on_m = wide and H_q // H_kv == 64   # 64 heads: the keys-on-M form of that kernel
     ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition,
                                                           sliding_window=window), 16),
                      dtype=torch.uint8, device=dev)
@@ -306,7 +310,8 @@ def build_decode(args, cfg, dev, rank):
     kv, alg = decode_bytes(ctx, B, H_q, H_kv, d, dt, window)
     # this library's kernels per layer: the append (3 for quantized pools), the decode and, when a
     # context spans several partitions, the split-K merge
-    parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, sliding_window=window) > 0
+    parts = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition,
+                                             sliding_window=window) > 0
     launches = L * ((3 if quant else 1) + 1 + (1 if parts else 0))
 
     # host-buffer (e2e) step: inputs from pinned memory, every layer's output read back
@@ -371,7 +376,8 @@ def build_decode(args, cfg, dev, rank):
                        f"events); each decode "
                        f"call reads {kv / 1e9:.2f} GB of K/V"),
                 "partition_tokens": args.partition or "auto", "sliding_window": window or None,
-                "decode_engine": {0: "tensor cores (tcgen05)" if wide else "tensor cores (mma.sync)",
+                "decode_engine": {0: ("tensor cores (tcgen05, keys on the MMA's M side)" if keys_on_m else
+                                      "tensor cores (tcgen05)") if wide else "tensor cores (mma.sync)",
                                   1: "tensor cores (mma.sync)", 2: "CUDA cores, packed fp32x2 FMA",
                                   3: "CUDA cores, fp32 FMA"}[args.engine]},
         kv_bytes_per_step=kv * L, layers=L,
@@ -380,7 +386,8 @@ def build_decode(args, cfg, dev, rank):
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
                       traffic=kernel_traffic(f"decode_{args.workload}",
-                                             DECODEQ_SRCS if quant else DECODETC_SRCS if wide else DECODE16_SRCS)),
+                                             DECODEQ_SRCS if quant else DECODETCK_SRCS if keys_on_m else
+                                             DECODETC_SRCS if wide else DECODE16_SRCS)),
         launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",
         h2d=h2d_bytes, d2h=d2h_bytes, calls_per_step=L, flush_l2=L == 1)
     return step, e2e_step, info, pool

@@ -454,6 +454,22 @@ namespace {
 
 constexpr int kStages = 2;
 
+// Groups of 64 query heads go to the keys-on-M tcgen05 kernel (decode_tc_keys.cu); 0 sends
+// them to the two-sequences-per-CTA one (decode_tc.cu).
+#ifndef PKV_DECODE_KEYS_TC
+#define PKV_DECODE_KEYS_TC 1
+#endif
+constexpr bool kDecodeKeysTc = PKV_DECODE_KEYS_TC != 0;
+
+}  // namespace
+
+bool decode_keys_tc_available(int d, int G, int kv_dtype)
+{
+    return kDecodeKeysTc && decode_tck_supported(d, G, kv_dtype);
+}
+
+namespace {
+
 template <typename K>
 int launch_k(K kernel, int smem, dim3 grid, int threads, cudaStream_t s, const DecodeParams& p,
              const CUtensorMap* tmk, const CUtensorMap* tmv)
@@ -530,6 +546,13 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
             return PKV_ERR_UNSUPPORTED;
         rc = launch_decode_simt(p, a.kv_dtype, a.G, a.engine == 2, grid, s, tmk, tmv);
+    } else if (kDecodeKeysTc && a.engine == 0 && a.window == 0 && a.part_base == 0 &&
+               decode_tck_supported(a.d, a.G, a.kv_dtype) && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
+        // 64 query heads per KV head: tcgen05 with the keys on the MMA's M side
+        CUtensorMap tmq;
+        auto enc = tensor_map_encoder();
+        if (!enc || !make_q_map_seq(&tmq, a.q, a.B, a.H_q, enc)) return PKV_ERR_CUDA;
+        rc = launch_decode_tck(p, a.kv_dtype, &tmq, tmk, tmv, s);
     } else if ((a.kv_dtype == PKV_BF16 || a.kv_dtype == PKV_F16) && a.engine == 0 && a.window == 0 &&
                a.part_base == 0 && decode_tc_supported(a.d, a.G, a.kv_dtype) &&
                (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {

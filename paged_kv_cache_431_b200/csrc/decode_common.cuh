@@ -98,6 +98,12 @@ bool decode_tc_supported(int d, int G, int kv_dtype);
 int launch_decode_tc(const DecodeParams& p, int kv_dtype, const CUtensorMap* tmq, const CUtensorMap* tmk,
                      const CUtensorMap* tmv, cudaStream_t s);
 
+// tcgen05 decode for groups of 64 query heads with the keys on the MMA's M side (decode_tc_keys.cu).
+bool decode_tck_supported(int d, int G, int kv_dtype);
+bool make_q_map_seq(CUtensorMap* map, const void* q, int B, int H_q, PFN_encode enc);
+int launch_decode_tck(const DecodeParams& p, int kv_dtype, const CUtensorMap* tmq, const CUtensorMap* tmk,
+                      const CUtensorMap* tmv, cudaStream_t s);
+
 // Launch the quantized-pool decode kernel (decode_quant.cu).
 int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,
                         const CUtensorMap* tmk, const CUtensorMap* tmv);

@@ -107,6 +107,10 @@ struct PrefillArgs {
 
 int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
 
+// The automatic decode engine for this shape is the keys-on-M tcgen05 kernel (decode_tc_keys.cu,
+// 64 query heads per KV head); its split-K partitions follow their own rule.
+bool decode_keys_tc_available(int d, int G, int kv_dtype);
+
 using PFN_encode = PFN_cuTensorMapEncodeTiled_v12000;
 PFN_encode tensor_map_encoder();   // null when no driver is present
 

@@ -23,10 +23,17 @@ __device__ __forceinline__ uint64_t sdesc_mn128(uint32_t addr, uint32_t lbo_byte
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// Instruction descriptor of kind::f16 with fp32 accumulation: A and B both bf16 or both f16,
+// each K-major or MN-major (transposed), M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_ab(bool bf16, bool a_mn_major, bool b_mn_major, int M, int N)
+{
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, bool b_mn_major, int M, int N)
 {
-    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    return idesc_f16_ab(bf16, false, b_mn_major, M, N);
 }
 
 __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate)

@@ -227,6 +227,24 @@ def test_decode_workspace_small_batches_and_explicit_partitions():
         pkv.lib().kv_pool_destroy(h)
 
 
+def test_decode_workspace_of_the_keys_on_m_engine():
+    """64 query heads per KV head (16-bit pools, d = 128, engine auto) run on the keys-on-M tcgen05
+    kernel, one CTA per SM: as few partitions per sequence as fill 148 SMs, each at most 4096
+    tokens in whole 128-key tiles; engine 1, other group sizes and explicit sizes keep the general rule."""
+    rc, h = _create(num_kv_heads=1, head_dim=128, kv_dtype=pkv.BF16)
+    assert rc == 0
+    try:
+        assert _decode_ws(h, 256, 64, 4096) == 0                              # one 4096-token partition
+        assert _decode_ws(h, 256, 64, 8000) == _ws_expected(256, 64, 1, 2)    # two of 4096 tokens
+        assert _decode_ws(h, 4, 64, 4096) == _ws_expected(4, 64, 1, 32)       # 4 sequences: 37 wanted, 128-token floor
+        assert _decode_ws(h, 100, 64, 1000) == _ws_expected(100, 64, 1, 2)    # 2 x 512 tokens fill 148 SMs
+        assert _decode_ws(h, 256, 64, 4096, pkv._DecodeOpts(1, 0, 0)) == _ws_expected(256, 64, 1, 8)   # engine 1: 512
+        assert _decode_ws(h, 256, 64, 4096, pkv._DecodeOpts(0, 1024, 0)) == _ws_expected(256, 64, 1, 4)
+        assert _decode_ws(h, 256, 128, 4096) == _ws_expected(256, 128, 1, 8)  # G = 128: the general rule
+    finally:
+        pkv.lib().kv_pool_destroy(h)
+
+
 def test_wait_hook_arguments_are_checked_on_the_host():
     """pkv_test_withhold_copy only stores process-wide settings; out-of-range bounds are
     rejected and tile < 0 restores the defaults (no CUDA call)."""
