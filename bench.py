@@ -54,6 +54,9 @@ DECODETC_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc.cu", "paged_kv_cache_43
 DECODETCK_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc_keys.cu", "paged_kv_cache_431_b200/csrc/tcgen05.cuh",
                   "paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                   "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
+DECODEQ8TC_SRCS = ["paged_kv_cache_431_b200/csrc/decode_tc_fp8.cu", "paged_kv_cache_431_b200/csrc/tcgen05.cuh",
+                   "paged_kv_cache_431_b200/csrc/decode.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
+                   "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 DECODEQ_SRCS = ["paged_kv_cache_431_b200/csrc/decode_quant.cu", "paged_kv_cache_431_b200/csrc/decode_common.cuh",
                 "paged_kv_cache_431_b200/csrc/common.cuh", "paged_kv_cache_431_b200/csrc/api.cu"]
 PREFILL_SRCS = ["paged_kv_cache_431_b200/csrc/prefill_tc.cu", "paged_kv_cache_431_b200/csrc/common.cuh"]
@@ -289,6 +292,8 @@ def build_decode(args, cfg, dev, rank):
     # per KV head (16-bit pool, head dim 128, no window)
     wide = not quant and d == 128 and H_q // H_kv in (64, 128) and not window and args.engine == 0
     keys_on_m = wide and H_q // H_kv == 64   # 64 heads: the keys-on-M form of that kernel
+    # fp8 pools with 8 query heads per KV head: the tcgen05 kernel that multiplies the e4m3 codes
+    fp8_tc = dt == wl.FP8 and d == 128 and H_q // H_kv == 8 and not window and args.engine == 0
     ws = torch.empty(max(pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, partition_tokens=args.partition,
                                                           sliding_window=window), 16),
                      dtype=torch.uint8, device=dev)
@@ -377,7 +382,9 @@ def build_decode(args, cfg, dev, rank):
                        f"call reads {kv / 1e9:.2f} GB of K/V"),
                 "partition_tokens": args.partition or "auto", "sliding_window": window or None,
                 "decode_engine": {0: ("tensor cores (tcgen05, keys on the MMA's M side)" if keys_on_m else
-                                      "tensor cores (tcgen05)") if wide else "tensor cores (mma.sync)",
+                                      "tensor cores (tcgen05)") if wide else
+                                     "tensor cores (tcgen05 kind::f8f6f4 on the e4m3 codes)" if fp8_tc else
+                                     "tensor cores (mma.sync)",
                                   1: "tensor cores (mma.sync)", 2: "CUDA cores, packed fp32x2 FMA",
                                   3: "CUDA cores, fp32 FMA"}[args.engine]},
         kv_bytes_per_step=kv * L, layers=L,
@@ -386,6 +393,7 @@ def build_decode(args, cfg, dev, rank):
                       peak=float(peaks["hbm_gbs"]), unit="GB/s",
                       peak_source=f"{kind} (MEASURED_PEAKS.json hbm_gbs)",
                       traffic=kernel_traffic(f"decode_{args.workload}",
+                                             DECODEQ8TC_SRCS if fp8_tc else
                                              DECODEQ_SRCS if quant else DECODETCK_SRCS if keys_on_m else
                                              DECODETC_SRCS if wide else DECODE16_SRCS)),
         launches_per_step=launches, dtype=DTYPE_NAME[dt] if quant else "bf16",

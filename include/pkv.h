@@ -166,16 +166,19 @@ PKV_API int kv_append(pkv_pool_t pool, int layer, const void* k, const void* v, 
 /* Tuning options for paged_decode_attn (NULL = defaults). */
 typedef struct {
     int32_t engine;            /* 0 auto: the 5th-generation tensor cores (tcgen05, TMEM accumulators)
-                                  for 16-bit pools with head_dim 128, G = 64 or 128 query heads per KV
-                                  head, no sliding window and a 16-byte-aligned q; engine 1 otherwise.
+                                  for head_dim 128, no sliding window and a 16-byte-aligned q with
+                                  16-bit pools and G = 64 or 128 query heads per KV head, or fp8 pools
+                                  and G = 8 (the e4m3 codes go to the MMA as they are); engine 1 otherwise.
                                   1 warp-level tensor cores (mma.sync), every pool dtype and group size.
                                   2 CUDA-core FP32 FMA with packed fp32x2 pairs, 3 CUDA-core scalar FP32 FMA:
                                   16-bit pools, head_dim 128, G 4 or 8, q 16-byte aligned (else
                                   PKV_ERR_UNSUPPORTED); kept to measure the FP32-pipe form of the decode */
     int32_t partition_tokens;  /* tokens per split-K partition; 0 = chosen from the workload (~256 KiB
                                   of K + V for 16-bit pools, ~192 KiB for quantized ones, fewer
-                                  tokens when the batch alone cannot fill the GPU); else a multiple of
-                                  16 in [64, 4096] (PKV_ERR_ARG otherwise) */
+                                  tokens when the batch alone cannot fill the GPU; on the tcgen05
+                                  engines for G = 64 (16-bit) and G = 8 (fp8): as few partitions per
+                                  sequence as fill the GPU, at most 4096 tokens, whole 128-token
+                                  tiles); else a multiple of 16 in [64, 4096] (PKV_ERR_ARG otherwise) */
     int32_t sliding_window;    /* 0 = attend to the whole context; w > 0 = sliding-window attention
                                   ([KVB] "The KV cache": sliding-window or local attention layers):
                                   the query (position context_len - 1) sees only positions

@@ -318,12 +318,12 @@ static int ctas_per_partition(pkv_pool_t pool, int num_q_heads)
     return H_kv * ((G + 15) / 16);
 }
 
-// Partition of the keys-on-M tcgen05 decode (one CTA per SM, a fixed cost per CTA): as few
-// partitions per sequence as fill the SMs, each at most 4096 tokens, in whole 128-key tiles.
-static int keys_tc_partition(int seq_heads, int span)
+// Partition of the keys-on-M tcgen05 decodes (one or two CTAs per SM, a fixed cost per CTA): as
+// few partitions per sequence as fill the SMs, each at most 4096 tokens, in whole 128-key tiles.
+static int keys_tc_partition(int seq_heads, int span, int ctas_per_sm)
 {
     int parts = (span + 4095) / 4096;
-    const int fill = (num_sms() + seq_heads - 1) / (seq_heads > 0 ? seq_heads : 1);
+    const int fill = (ctas_per_sm * num_sms() + seq_heads - 1) / (seq_heads > 0 ? seq_heads : 1);
     parts = parts < fill ? fill : parts;
     parts = parts < 1 ? 1 : parts;
     const int P = ((span + parts - 1) / parts + 127) / 128 * 128;
@@ -338,10 +338,11 @@ static int decode_partitioning(pkv_pool_t pool, int num_seqs, int num_q_heads, i
     // with a window a sequence's partitions start at the block holding ctx - window
     const int span = (window > 0 && max_ctx > window + PKV_BLOCK_SIZE - 1) ? window + PKV_BLOCK_SIZE - 1 : max_ctx;
     const int H_kv = pool->d.num_kv_heads;
-    const bool keys_tc = (!opts || opts->engine == 0) && window == 0 && num_q_heads % H_kv == 0 &&
-                         decode_keys_tc_available(pool->d.head_dim, num_q_heads / H_kv, pool->d.kv_dtype);
-    if (keys_tc && !(opts && opts->partition_tokens > 0))
-        *P = keys_tc_partition(num_seqs * H_kv, span);
+    const int keys_tc = ((!opts || opts->engine == 0) && window == 0 && num_q_heads % H_kv == 0)
+                            ? decode_keys_tc_available(pool->d.head_dim, num_q_heads / H_kv, pool->d.kv_dtype)
+                            : 0;
+    if (keys_tc > 0 && !(opts && opts->partition_tokens > 0))
+        *P = keys_tc_partition(num_seqs * H_kv, span, keys_tc);
     else
         *P = choose_partition(num_seqs, ctas_per_partition(pool, num_q_heads), span, pool->row_bytes,
                               is_quantized(pool->d.kv_dtype), opts);

@@ -461,11 +461,20 @@ constexpr int kStages = 2;
 #endif
 constexpr bool kDecodeKeysTc = PKV_DECODE_KEYS_TC != 0;
 
+// fp8 pools with 8 query heads per KV head go to the tcgen05 kernel that multiplies the stored
+// codes (decode_tc_fp8.cu); 0 sends them to the warp-level one (decode_quant.cu).
+#ifndef PKV_DECODE_TC_FP8
+#define PKV_DECODE_TC_FP8 1
+#endif
+constexpr bool kDecodeTcFp8 = PKV_DECODE_TC_FP8 != 0;
+
 }  // namespace
 
-bool decode_keys_tc_available(int d, int G, int kv_dtype)
+int decode_keys_tc_available(int d, int G, int kv_dtype)
 {
-    return kDecodeKeysTc && decode_tck_supported(d, G, kv_dtype);
+    if (kDecodeKeysTc && decode_tck_supported(d, G, kv_dtype)) return 1;
+    if (kDecodeTcFp8 && decode_tc_fp8_supported(d, G, kv_dtype)) return 2;
+    return 0;
 }
 
 namespace {
@@ -546,6 +555,10 @@ int launch_decode(const DecodeArgs& a, const CUtensorMap* tmk, const CUtensorMap
         if (!decode_simt_supported(a.d, a.G, a.kv_dtype) || (reinterpret_cast<uintptr_t>(a.q) & 15))
             return PKV_ERR_UNSUPPORTED;
         rc = launch_decode_simt(p, a.kv_dtype, a.G, a.engine == 2, grid, s, tmk, tmv);
+    } else if (kDecodeTcFp8 && a.engine == 0 && a.window == 0 && a.part_base == 0 &&
+               decode_tc_fp8_supported(a.d, a.G, a.kv_dtype) && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
+        // fp8 pools, 8 query heads per KV head: the codes go to tcgen05 kind::f8f6f4 MMAs
+        rc = launch_decode_tc_fp8(p, tmk, tmv, s);
     } else if (kDecodeKeysTc && a.engine == 0 && a.window == 0 && a.part_base == 0 &&
                decode_tck_supported(a.d, a.G, a.kv_dtype) && (reinterpret_cast<uintptr_t>(a.q) & 15) == 0) {
         // 64 query heads per KV head: tcgen05 with the keys on the MMA's M side

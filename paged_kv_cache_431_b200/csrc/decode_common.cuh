@@ -104,6 +104,11 @@ bool make_q_map_seq(CUtensorMap* map, const void* q, int B, int H_q, PFN_encode 
 int launch_decode_tck(const DecodeParams& p, int kv_dtype, const CUtensorMap* tmq, const CUtensorMap* tmk,
                       const CUtensorMap* tmv, cudaStream_t s);
 
+// tcgen05 decode for fp8 pools with 8 query heads per KV head, codes fed to kind::f8f6f4
+// MMAs (decode_tc_fp8.cu).
+bool decode_tc_fp8_supported(int d, int G, int kv_dtype);
+int launch_decode_tc_fp8(const DecodeParams& p, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
+
 // Launch the quantized-pool decode kernel (decode_quant.cu).
 int launch_decode_quant(const DecodeParams& p, int kv_dtype, int d, int nht, dim3 grid, cudaStream_t s,
                         const CUtensorMap* tmk, const CUtensorMap* tmv);

@@ -107,9 +107,11 @@ struct PrefillArgs {
 
 int launch_prefill(const PrefillArgs& a, const CUtensorMap* tmk, const CUtensorMap* tmv, cudaStream_t s);
 
-// The automatic decode engine for this shape is the keys-on-M tcgen05 kernel (decode_tc_keys.cu,
-// 64 query heads per KV head); its split-K partitions follow their own rule.
-bool decode_keys_tc_available(int d, int G, int kv_dtype);
+// CTAs per SM of the automatic decode engine for this shape when it is one of the keys-on-M
+// tcgen05 kernels (decode_tc_keys.cu: 64 query heads per KV head, one CTA per SM;
+// decode_tc_fp8.cu: fp8 pools with 8, two CTAs per SM), else 0.  Their split-K partitions
+// follow their own rule.
+int decode_keys_tc_available(int d, int G, int kv_dtype);
 
 using PFN_encode = PFN_cuTensorMapEncodeTiled_v12000;
 PFN_encode tensor_map_encoder();   // null when no driver is present

@@ -184,12 +184,12 @@ def _ws_expected(B, H_q, H_kv, parts, d=128):
     return B * H_q * parts * (d + 2) * 4
 
 
-@pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 768), (pkv.FP8E4M3, 768),
-                                     (pkv.INT4, 1536)])
+@pytest.mark.parametrize("dtype,P", [(pkv.BF16, 512), (pkv.F16, 512), (pkv.INT8, 768), (pkv.INT4, 1536)])
 def test_decode_workspace_follows_the_partition_policy(dtype, P):
     """Split-K partitions of ~256 KiB of K + V for 16-bit pools and ~192 KiB for quantized ones (512 /
     768 / 1536 tokens at d = 128) when the batch fills the GPU; the workspace is fp32 o[d] + (m, l)
-    per (sequence, query head, partition)."""
+    per (sequence, query head, partition).  (fp8 pools with 8 query heads per KV head run on the
+    tcgen05 kernel and its own rule: test_decode_workspace_of_the_keys_on_m_engines.)"""
     kw = dict(num_kv_heads=8, head_dim=128, kv_dtype=dtype)
     if dtype in pkv.QUANTIZED:
         kw.update(k_scale=0x30000, v_scale=0x40000)
@@ -227,10 +227,11 @@ def test_decode_workspace_small_batches_and_explicit_partitions():
         pkv.lib().kv_pool_destroy(h)
 
 
-def test_decode_workspace_of_the_keys_on_m_engine():
+def test_decode_workspace_of_the_keys_on_m_engines():
     """64 query heads per KV head (16-bit pools, d = 128, engine auto) run on the keys-on-M tcgen05
     kernel, one CTA per SM: as few partitions per sequence as fill 148 SMs, each at most 4096
-    tokens in whole 128-key tiles; engine 1, other group sizes and explicit sizes keep the general rule."""
+    tokens in whole 128-key tiles; engine 1, other group sizes and explicit sizes keep the general
+    rule.  fp8 pools with 8 query heads per KV head: the same rule with two CTAs per SM."""
     rc, h = _create(num_kv_heads=1, head_dim=128, kv_dtype=pkv.BF16)
     assert rc == 0
     try:
@@ -241,6 +242,16 @@ def test_decode_workspace_of_the_keys_on_m_engine():
         assert _decode_ws(h, 256, 64, 4096, pkv._DecodeOpts(1, 0, 0)) == _ws_expected(256, 64, 1, 8)   # engine 1: 512
         assert _decode_ws(h, 256, 64, 4096, pkv._DecodeOpts(0, 1024, 0)) == _ws_expected(256, 64, 1, 4)
         assert _decode_ws(h, 256, 128, 4096) == _ws_expected(256, 128, 1, 8)  # G = 128: the general rule
+    finally:
+        pkv.lib().kv_pool_destroy(h)
+    rc, h = _create(num_kv_heads=8, head_dim=128, kv_dtype=pkv.FP8E4M3, k_scale=0x30000, v_scale=0x40000)
+    assert rc == 0
+    try:
+        assert _decode_ws(h, 170, 64, 8192) == _ws_expected(170, 64, 8, 2)    # 2 x 4096 tokens
+        assert _decode_ws(h, 16, 64, 131072) == _ws_expected(16, 64, 8, 32)   # the long-context layer
+        assert _decode_ws(h, 4, 64, 4096) == _ws_expected(4, 64, 8, 8)        # 10 parts wanted, 410 -> 512 tokens: 8
+        assert _decode_ws(h, 16, 64, 131072, pkv._DecodeOpts(1, 0, 0)) == _ws_expected(16, 64, 8, 171)   # engine 1: 768
+        assert _decode_ws(h, 16, 32, 131072) == _ws_expected(16, 32, 8, 171)  # G = 4: the general rule
     finally:
         pkv.lib().kv_pool_destroy(h)
 

@@ -119,6 +119,8 @@ DECODE_CASES = [
     (32, 4, 128, 0),      # G = 8
     (32, 2, 128, 128),    # G = 16
     (12, 4, 64, 64),      # G = 3
+    (32, 4, 128, 128),    # G = 8, split-K over one-tile partitions
+    (16, 2, 128, 256),    # G = 8, two tiles per partition
 ]
 
 

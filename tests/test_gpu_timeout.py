@@ -58,6 +58,7 @@ DECODES = {
     "int4": (32, 4, wl.INT4, pkv.ENGINE_MMA, 64),
     "cuda_cores": (32, 4, wl.BF16, pkv.ENGINE_FMA2, 64),
     "tcgen05_g64": (64, 1, wl.BF16, pkv.ENGINE_AUTO, 256),
+    "tcgen05_fp8": (32, 4, wl.FP8, pkv.ENGINE_AUTO, 256),
 }
 
 
