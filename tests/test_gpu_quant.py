@@ -154,6 +154,34 @@ def test_quantized_decode_parity(dt, case):
     assert torch.all(out[0] == 0)
 
 
+@pytest.mark.parametrize("H_q", [64, 32])
+@pytest.mark.parametrize("dt", QDTYPES, ids=lambda x: NAMES[x])
+def test_quantized_decode_fp16_query(dt, H_q):
+    """q in fp16 instead of bf16 (both are accepted for quantized pools): 8 query heads per KV
+    head (for fp8 the tcgen05 kernel, which reads q itself) and 4 (the warp-level kernel), with
+    split-K partitions, against the oracle given the same fp16 q."""
+    H_kv, d = 8, 128
+    g = wl.generator(1300 + dt + H_q)
+    lens = [1, 17, 200] + torch.randint(300, 900, (3,), generator=g).tolist()
+    N = sum(wl.ceil_div(n, 16) for n in lens) + 2
+    paging = wl.allocate(lens, N, 64, g)
+    pool = pkv.KVPool.allocate(1, N, H_kv, d, dt)
+    opool = oracle_copy(pool)
+    seq = torch.cat([torch.full((n,), b) for b, n in enumerate(lens)])
+    pos = torch.cat([torch.arange(n) for n in lens])
+    slots = wl.slots_for(paging.tables, seq, pos)
+    k, v = wl.kv_source(len(seq), H_kv, d, g)
+    pkv.kv_append(pool, 0, k.to(DEV), v.to(DEV), slots.to(DEV))
+    oracle.kv_append(opool, k, v, oracle.BF16, slots.numpy())
+    q = wl.normal((len(lens), H_q, d), torch.float16, g)
+    out = pkv.paged_decode_attn(pool, 0, q.to(DEV), paging.tables.to(DEV), paging.ctx_lens.to(DEV), d ** -0.5,
+                                max(lens), partition_tokens=256)
+    torch.cuda.synchronize()
+    assert pkv.read_device_status(pool) == 0
+    ref = oracle.paged_decode(opool, q, oracle.F16, paging.tables, paging.ctx_lens, np.float32(d ** -0.5))
+    assert max_abs_diff(out, ref) <= TOL
+
+
 @pytest.mark.parametrize("dt", QDTYPES, ids=lambda x: NAMES[x])
 def test_quantized_long_context_config(dt):
     """Quantized long-context decode, 1 layer: B 16, H_q 64, H_kv 8, d 128, contexts
