@@ -36,19 +36,20 @@ def decode_inputs(seed, B, H_q, H_kv, d, kv_dtype=wl.BF16):
 
 
 CASES = {
-    # name: (pool dtype, sliding window)
-    "bf16": (wl.BF16, 0),
-    "int8": (wl.INT8, 0),
-    "bf16_window": (wl.BF16, 1000),
+    # name: (pool dtype, sliding window, query heads (8 KV heads), batches of the two calls)
+    "bf16": (wl.BF16, 0, 32, (64, 24)),
+    "int8": (wl.INT8, 0, 32, (64, 24)),
+    "bf16_window": (wl.BF16, 1000, 32, (64, 24)),
+    "fp8_g8": (wl.FP8, 0, 64, (24, 8)),   # 8 query heads per KV head: the tcgen05 fp8 kernel
 }
 
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_noalloc_matches_regular_decode_on_two_calls(name):
-    kv_dtype, window = CASES[name]
-    for seed, B in ((801, 64), (802, 24)):
-        pool, q, tables, ctx, max_ctx = decode_inputs(seed, B, 32, 8, 128, kv_dtype)
-        need = pkv.paged_decode_workspace_bytes(pool, B, 32, max_ctx, sliding_window=window)
+    kv_dtype, window, H_q, batches = CASES[name]
+    for seed, B in zip((801, 802), batches):
+        pool, q, tables, ctx, max_ctx = decode_inputs(seed, B, H_q, 8, 128, kv_dtype)
+        need = pkv.paged_decode_workspace_bytes(pool, B, H_q, max_ctx, sliding_window=window)
         assert 0 < need <= pkv.NOALLOC_SCRATCH_BYTES          # the split-K path is exercised
         ref = pkv.paged_decode_attn(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx, sliding_window=window)
         out = pkv.paged_decode_attn_noalloc(pool, 0, q, tables, ctx, 128 ** -0.5, max_ctx, sliding_window=window)
